@@ -1,0 +1,79 @@
+// Host-side internals shared by the translation units of libsvdq: the
+// prepared-weights handle, layout helpers and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/svdq.h"
+
+namespace svdq {
+
+constexpr int kRankMax = 64;
+
+inline int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+inline int rank_pad_of(int rank) { return rank == 0 ? 0 : static_cast<int>(round_up(rank, 32)); }
+inline int64_t n_pad_of(int64_t n) { return round_up(n, 256); }
+inline int64_t m_pad_of(int64_t m) { return round_up(m, 128); }
+
+// Byte size of the scale buffer for `rows` rows (rows padded per precision).
+inline size_t nvfp4_scale_bytes(int64_t rows_padded, int K) { return static_cast<size_t>(rows_padded) * (K / 16); }
+inline size_t int4_scale_bytes(int64_t rows_padded, int K) { return static_cast<size_t>(rows_padded) * (K / 64) * 2; }
+
+// Offsets (bytes) of the sub-buffers inside the caller's weight storage.
+struct WeightLayout {
+  size_t qw, sw, l1s, l2, inv_lambda, bias, status, amax, total;
+  size_t sw_bytes;
+};
+WeightLayout weight_layout(const svdq_layer_desc& d);
+
+}  // namespace svdq
+
+// The opaque handle of the C ABI.
+struct svdq_weights {
+  svdq_layer_desc desc;
+  int rank_pad;
+  int64_t n_pad;
+  float g_w;
+  uint8_t* base;  // caller's storage
+  uint8_t* qw;
+  void* sw;
+  size_t sw_bytes;
+  uint16_t* l1s;
+  float* l2;
+  float* inv_lambda;
+  float* bias;
+  int* status;    // written by GEMM kernels when a bounded wait runs out
+  uint32_t* amax; // scratch word of the preparation pass
+  int device;
+  CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes
+  CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes
+};
+
+namespace svdq {
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_smoothing_lambda(const uint16_t* X, int M, const float* W, int N, int K, float* lambda,
+                                    float* scratch, cudaStream_t s);
+cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* lambda, const uint16_t* L1,
+                           const uint16_t* L2, const uint16_t* bias, cudaStream_t s);
+cudaError_t launch_act_global_scale(const svdq_weights* w, const uint16_t* X, int M, float* g_x, cudaStream_t s);
+cudaError_t launch_quantize(const svdq_weights* w, const uint16_t* X, int M, float g_x, uint8_t* qx, void* sx,
+                            float* lora_act, cudaStream_t s);
+cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
+                              const float* lora_act, int M, void* Y, int out_dtype, cudaStream_t s);
+cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* lora_act, int M,
+                             void* Y, int out_dtype, cudaStream_t s);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).  2-D, row-major, `inner` elements per
+// row of `row_bytes` stride, box {box_inner, box_rows}, 128-byte swizzle.
+bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
+
+int num_sms(int device);
+
+}  // namespace svdq

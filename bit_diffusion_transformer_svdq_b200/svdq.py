@@ -1,0 +1,230 @@
+"""Thin Python binding of libsvdq (include/svdq.h).
+
+Argument marshalling only: tensors are passed as device pointers, streams as
+cudaStream_t handles; every step of the layer runs in the library's CUDA
+kernels.  The functions keep the C names.  A missing library is an error
+(there is no fallback path).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+SVDQ_NVFP4 = 0
+SVDQ_INT4 = 1
+SVDQ_OUT_BF16 = 0
+SVDQ_OUT_F32 = 1
+
+STATUS_NAMES = {
+    0: "SVDQ_OK",
+    1: "SVDQ_ERR_INVALID_ARG",
+    2: "SVDQ_ERR_SHAPE",
+    3: "SVDQ_ERR_ALIGNMENT",
+    4: "SVDQ_ERR_UNSUPPORTED_DEVICE",
+    5: "SVDQ_ERR_CUDA",
+    6: "SVDQ_ERR_TIMEOUT",
+    7: "SVDQ_ERR_WORKSPACE",
+}
+
+
+class SVDQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        super().__init__(f"{where}: {STATUS_NAMES.get(self.status, self.status)} ({svdq_status_string(self.status)})")
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("precision", ctypes.c_int32), ("group_size", ctypes.c_int32)]
+
+
+class WeightsView(ctypes.Structure):
+    _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("rank", ctypes.c_int32), ("rank_pad", ctypes.c_int32),
+                ("precision", ctypes.c_int32), ("group_size", ctypes.c_int32), ("n_pad", ctypes.c_int32),
+                ("g_w", ctypes.c_float), ("qw", ctypes.c_void_p), ("sw", ctypes.c_void_p),
+                ("sw_bytes", ctypes.c_size_t), ("l1s", ctypes.c_void_p), ("l2", ctypes.c_void_p),
+                ("inv_lambda", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
+
+
+_lib = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+_SIGS = {
+    "svdq_status_string": (ctypes.c_char_p, [_I]),
+    "svdq_check_device": (_I, [ctypes.c_int]),
+    "svdq_smoothing_lambda": (_I, [_P, _I, _P, _I, _I, _P, _P, _P]),
+    "svdq_weights_bytes": (_Z, [ctypes.POINTER(LayerDesc)]),
+    "svdq_prepare_weights": (_I, [ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P, _Z, ctypes.POINTER(_P), _P]),
+    "svdq_weights_destroy": (None, [_P]),
+    "svdq_weights_get_view": (_I, [_P, ctypes.POINTER(WeightsView)]),
+    "svdq_act_global_scale": (_I, [_P, _P, _I, _P, _P]),
+    "svdq_act_scale_bytes": (_Z, [_P, _I]),
+    "svdq_quantize_act_lora_down": (_I, [_P, _P, _I, _F, _P, _P, _P, _P]),
+    "svdq_w4a4_gemm_lora_up": (_I, [_P, _P, _P, _F, _P, _I, _P, _I, _P]),
+    "svdq_workspace_bytes": (_Z, [_P, _I]),
+    "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
+    "svdq_device_status": (_I, [_P, _P]),
+}
+
+
+def load_library() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libsvdq.so is not built ({LIB_PATH}); run `python -m bit_diffusion_transformer_svdq_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SVDQError(status, where)
+
+
+def svdq_status_string(status: int) -> str:
+    return load_library().svdq_status_string(int(status)).decode()
+
+
+def svdq_check_device(device: int = 0) -> int:
+    return load_library().svdq_check_device(int(device))
+
+
+def make_desc(K: int, N: int, rank: int, precision: int = SVDQ_NVFP4) -> LayerDesc:
+    return LayerDesc(K, N, rank, precision, 16 if precision == SVDQ_NVFP4 else 64)
+
+
+def svdq_weights_bytes(desc: LayerDesc) -> int:
+    return load_library().svdq_weights_bytes(ctypes.byref(desc))
+
+
+def svdq_smoothing_lambda(X: torch.Tensor, W: torch.Tensor, lam: torch.Tensor, scratch: torch.Tensor, stream=None):
+    M, K = X.shape
+    N = W.shape[0]
+    _check(load_library().svdq_smoothing_lambda(_ptr(X), M, _ptr(W), N, K, _ptr(lam), _ptr(scratch), _stream(stream)),
+           "svdq_smoothing_lambda")
+
+
+class Weights:
+    """Owns the host handle of prepared weights and keeps the caller's
+    device storage tensor alive alongside it."""
+
+    def __init__(self, handle: int, storage: torch.Tensor, desc: LayerDesc):
+        self.handle = handle
+        self.storage = storage
+        self.desc = desc
+
+    @property
+    def _as_parameter_(self):
+        return self.handle
+
+    def view(self) -> WeightsView:
+        v = WeightsView()
+        _check(load_library().svdq_weights_get_view(self.handle, ctypes.byref(v)), "svdq_weights_get_view")
+        return v
+
+    def close(self) -> None:
+        if self.handle:
+            load_library().svdq_weights_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def svdq_prepare_weights(desc: LayerDesc, W, lam, L1, L2, bias, storage: torch.Tensor, stream=None) -> Weights:
+    out = ctypes.c_void_p()
+    _check(load_library().svdq_prepare_weights(ctypes.byref(desc), _ptr(W), _ptr(lam), _ptr(L1), _ptr(L2), _ptr(bias),
+                                               _ptr(storage), storage.numel() * storage.element_size(),
+                                               ctypes.byref(out), _stream(stream)), "svdq_prepare_weights")
+    return Weights(out.value, storage, desc)
+
+
+def svdq_act_global_scale(w: Weights, X: torch.Tensor, g_x: torch.Tensor, stream=None) -> None:
+    _check(load_library().svdq_act_global_scale(w.handle, _ptr(X), X.shape[0], _ptr(g_x), _stream(stream)),
+           "svdq_act_global_scale")
+
+
+def svdq_act_scale_bytes(w: Weights, M: int) -> int:
+    return load_library().svdq_act_scale_bytes(w.handle, M)
+
+
+def svdq_workspace_bytes(w: Weights, M: int) -> int:
+    return load_library().svdq_workspace_bytes(w.handle, M)
+
+
+def svdq_quantize_act_lora_down(w: Weights, X, M: int, g_x: float, qx, sx, lora_act, stream=None) -> None:
+    _check(load_library().svdq_quantize_act_lora_down(w.handle, _ptr(X), M, float(g_x), _ptr(qx), _ptr(sx),
+                                                      _ptr(lora_act), _stream(stream)), "svdq_quantize_act_lora_down")
+
+
+def svdq_w4a4_gemm_lora_up(w: Weights, qx, sx, g_x: float, lora_act, M: int, Y, out_dtype: int = SVDQ_OUT_BF16,
+                           stream=None) -> None:
+    _check(load_library().svdq_w4a4_gemm_lora_up(w.handle, _ptr(qx), _ptr(sx), float(g_x), _ptr(lora_act), M, _ptr(Y),
+                                                 out_dtype, _stream(stream)), "svdq_w4a4_gemm_lora_up")
+
+
+def svdq_linear_forward(w: Weights, X, M: int, g_x: float, Y, workspace, ws_bytes: int,
+                        out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    _check(load_library().svdq_linear_forward(w.handle, _ptr(X), M, float(g_x), _ptr(Y), out_dtype, _ptr(workspace),
+                                              ws_bytes, _stream(stream)), "svdq_linear_forward")
+
+
+def svdq_device_status(w: Weights, stream=None) -> int:
+    return load_library().svdq_device_status(w.handle, _stream(stream))
+
+
+# ----------------------------------------------------------------- helpers
+# Allocation-only conveniences (torch owns the device memory).
+
+def prepare_layer(W: torch.Tensor, lam: torch.Tensor, L1: torch.Tensor | None, L2: torch.Tensor | None,
+                  bias: torch.Tensor | None, rank: int, precision: int = SVDQ_NVFP4, stream=None) -> Weights:
+    """W (N x K fp32), lam (K fp32), L1 (rank x K bf16), L2 (N x rank bf16),
+    bias (N bf16), all on the current CUDA device."""
+    N, K = W.shape
+    desc = make_desc(K, N, rank, precision)
+    nbytes = svdq_weights_bytes(desc)
+    if nbytes == 0:
+        raise SVDQError(2, "svdq_weights_bytes")
+    storage = torch.empty(nbytes + 1024, dtype=torch.uint8, device=W.device)
+    off = (-storage.data_ptr()) % 1024
+    storage = storage[off:off + nbytes]
+    return svdq_prepare_weights(desc, W, lam, L1, L2, bias, storage, stream)
+
+
+def alloc_workspace(w: Weights, M: int, device) -> torch.Tensor:
+    n = svdq_workspace_bytes(w, M)
+    buf = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 1024
+    return buf[off:off + n]

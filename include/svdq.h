@@ -1,0 +1,215 @@
+/*
+ * svdq.h - C ABI of the B200 (sm_100a) SVDQuant W4A4 linear layer.
+ *
+ * What the layer computes (Nunchaku 4-bit quantisation in Diffusers,
+ * section "Nunchaku und SVDQuant"; charmloop.ai Nunchaku news item,
+ * second paragraph):
+ *
+ *     X_hat = X / lambda                 activation outliers moved into W
+ *     W_til = W * diag(lambda)
+ *     R     = W_til - (L1 L2)^T          residual of a 16-bit low-rank branch
+ *     Y     = X_hat L1 L2 + Q(X_hat) Q(R)^T + b
+ *
+ * Q() is 4-bit group quantisation: NVFP4 (E2M1 values, one E4M3 scale per
+ * 16 values, one fp32 tensor scale) or INT4 (one fp16 scale per 64 values);
+ * the precision / group_size / rank triple is the svdq_w4a4 block of the
+ * page's quantization_config ("Native Ladefunktion").  The lora-down
+ * X_hat L1 runs inside the activation-quantisation kernel and the lora-up
+ * inside the 4-bit GEMM, as the news item describes.
+ *
+ * Conventions for every entry point:
+ *   - Matrices are row-major.  "bf16" buffers hold raw bfloat16 bit
+ *     patterns in uint16_t.  Orientation follows nn.Linear: X is M x K,
+ *     W is N x K, Y is M x N.  L1 ("lora_down") is stored rank x K and
+ *     L2 ("lora_up") N x rank, so that the branch is X_hat L1^T L2^T.
+ *   - Every buffer is caller-owned.  Pointers marked [device] must be CUDA
+ *     device memory of the current device, 16-byte aligned; [host] pointers
+ *     are host memory.  The library never allocates device memory.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on that stream unless stated otherwise.
+ *   - Errors are returned as svdq_status; nothing aborts or exits.  Shape
+ *     and argument checks happen on the host before any launch.
+ *   - Only compute capability 10.0 (B200, sm_100a) is supported; other
+ *     devices get SVDQ_ERR_UNSUPPORTED_DEVICE (the pages' load-time GPU
+ *     capability check, "Hardware-Unterstuetzung").
+ *
+ * Shape limits: K % 64 == 0 (NVFP4: four 16-wide groups per MMA step;
+ * INT4: one 64-wide group), N % 16 == 0, 0 <= rank <= 64 with rank % 8 == 0,
+ * (precision, group_size) in {(NVFP4, 16), (INT4, 64)}, M >= 0.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer, bad enum, bad combination */
+  SVDQ_ERR_SHAPE = 2,              /* a size outside the limits above */
+  SVDQ_ERR_ALIGNMENT = 3,          /* a device pointer not 16-byte aligned */
+  SVDQ_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not compute capability 10.0 */
+  SVDQ_ERR_CUDA = 5,               /* a CUDA runtime call or launch failed */
+  SVDQ_ERR_TIMEOUT = 6,            /* a bounded wait inside a kernel ran out */
+  SVDQ_ERR_WORKSPACE = 7           /* storage / workspace smaller than required */
+} svdq_status;
+
+typedef enum svdq_precision {
+  SVDQ_NVFP4 = 0, /* E2M1 codes, E4M3 scale per 16, fp32 tensor scale */
+  SVDQ_INT4 = 1   /* signed 4-bit codes, fp16 scale per 64 */
+} svdq_precision;
+
+typedef enum svdq_out_dtype {
+  SVDQ_OUT_BF16 = 0, /* production output: bf16, round to nearest even */
+  SVDQ_OUT_F32 = 1   /* parity/debug output: the same epilogue stored in fp32 */
+} svdq_out_dtype;
+
+/* One quantised linear layer (the svdq_w4a4 block of quantization_config). */
+typedef struct svdq_layer_desc {
+  int32_t K;          /* input features */
+  int32_t N;          /* output features */
+  int32_t rank;       /* low-rank branch width r (0 = no branch) */
+  int32_t precision;  /* svdq_precision */
+  int32_t group_size; /* 16 for NVFP4, 64 for INT4 */
+} svdq_layer_desc;
+
+/* Opaque host handle of prepared weights.  The device data it refers to
+ * lives in the caller's `storage` buffer (see svdq_prepare_weights); the
+ * handle must not outlive that buffer. */
+typedef struct svdq_weights svdq_weights;
+
+/* Read-only view of prepared weights, for inspection and parity checks.
+ * All pointers are [device] and point into the caller's storage.
+ *   qw        N x K/2 bytes, two codes per byte, even k in the low nibble.
+ *             NVFP4: E2M1 nibbles (bit 3 = sign); INT4: two's complement.
+ *   sw        NVFP4: E4M3 bytes in the tiled scale layout (below) with
+ *             rows = N padded to a multiple of 256.
+ *             INT4: fp16, group-major: sw[g * n_pad + n], g < K/64.
+ *   l1s       rank_pad x K bf16: bf16(RN32(L1[t,k] * inv_lambda[k])),
+ *             rows t >= rank are zero.
+ *   l2        N x rank_pad fp32 copy of L2 (exact), columns t >= rank zero.
+ *   inv_lambda K fp32 = RN32(1 / lambda).
+ *   bias      N fp32 (widened from bf16; zeros when no bias was given).
+ *
+ * Tiled scale layout (NVFP4 sx and sw; the layout the tensor cores read):
+ * rows are padded to a multiple of 128 (256 for sw); the byte of row m and
+ * 16-wide group j (j < K/16) sits at
+ *     ((m / 128) * (K / 64) + j / 4) * 512 + (m % 32) * 16 + ((m / 32) % 4) * 4 + j % 4.
+ */
+typedef struct svdq_weights_view {
+  int32_t K, N, rank, rank_pad, precision, group_size;
+  int32_t n_pad;       /* scale rows: N rounded up to a multiple of 256 */
+  float g_w;           /* NVFP4 weight tensor scale (1 for INT4) */
+  const uint8_t* qw;
+  const void* sw;
+  size_t sw_bytes;
+  const uint16_t* l1s;
+  const float* l2;
+  const float* inv_lambda;
+  const float* bias;
+} svdq_weights_view;
+
+/* Human-readable name of a status code (static string). */
+SVDQ_API const char* svdq_status_string(svdq_status s);
+
+/* SVDQ_OK when `device` is a compute capability 10.0 GPU. */
+SVDQ_API svdq_status svdq_check_device(int device);
+
+/* Per-input-channel smoothing factor (the migration of activation outliers
+ * into the weights, "Nunchaku und SVDQuant"):
+ *     lambda[k] = RN32(sqrt(max_m |X[m,k]| / max_n |W[n,k]|)) in fp64,
+ *     lambda[k] = 1 when either maximum is 0.
+ * X [device] M x K bf16, W [device] N x K fp32, lambda [device] K fp32 out,
+ * scratch [device] 2*K fp32, overwritten.  M, N >= 1. */
+SVDQ_API svdq_status svdq_smoothing_lambda(const uint16_t* X, int32_t M, const float* W, int32_t N, int32_t K,
+                                  float* lambda, float* scratch, void* stream);
+
+/* Device bytes of the storage that svdq_prepare_weights fills. */
+SVDQ_API size_t svdq_weights_bytes(const svdq_layer_desc* desc);
+
+/* Weight preparation on the GPU (offline; the pages' quantiser step):
+ *   inv_lambda = RN32(1/lambda); W_til = RN32(W * lambda);
+ *   R[n,k] = RN32(fp64 chain W_til[n,k] - L1[0,k] L2[n,0] - ... - L1[r-1,k] L2[n,r-1]);
+ *   NVFP4: g_w = RN32(amax|R| / 2688) (1 if amax is 0), E4M3 scale per 16
+ *   and E2M1 codes by the rule of svdq_quantize_act_lora_down; INT4: fp16
+ *   scale per 64 and signed codes;  L1s = bf16(RN32(L1 * inv_lambda)).
+ * Inputs [device]: W N x K fp32, lambda K fp32, L1 rank x K bf16,
+ * L2 N x rank bf16, bias N bf16 or NULL.  L1/L2 may be NULL when rank == 0.
+ * storage [device] at least svdq_weights_bytes(desc) bytes, 1024-byte
+ * aligned, caller-owned; *out receives a host handle (free it with
+ * svdq_weights_destroy).  SYNCHRONOUS: returns after the GPU work is done
+ * (g_w is read back to the host). */
+SVDQ_API svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, const float* lambda,
+                                 const uint16_t* L1, const uint16_t* L2, const uint16_t* bias,
+                                 void* storage, size_t storage_bytes, svdq_weights** out, void* stream);
+
+/* Frees the host handle (not the caller's device storage).  NULL is a no-op. */
+SVDQ_API void svdq_weights_destroy(svdq_weights* w);
+
+SVDQ_API svdq_status svdq_weights_get_view(const svdq_weights* w, svdq_weights_view* view);
+
+/* Static activation tensor scale for NVFP4: g_x = RN32(amax |X_hat| / 2688)
+ * with X_hat = RN32(X * inv_lambda) (1 when amax is 0), written to
+ * g_x [device] (one fp32).  X [device] M x K bf16, M >= 1. */
+SVDQ_API svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t* X, int32_t M, float* g_x, void* stream);
+
+/* Bytes of the activation scale buffer sx for M rows:
+ * NVFP4: ceil(M/128)*128 * K/16 (tiled layout); INT4: 2 * K/64 * ceil(M/128)*128. */
+SVDQ_API size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M);
+
+/* Fused smoothing + 4-bit activation quantisation + lora-down (one pass
+ * over X).  For every row m and group:
+ *   x_hat = RN32(X[m,k] * inv_lambda[k])
+ *   NVFP4 (group 16, tensor scale g_x > 0):
+ *     s_q = E4M3_RNE_satfinite(RN32(RN32(amax/6) / g_x)), s = value(s_q);
+ *     s == 0 -> codes +0; else code = E2M1_RNE_satfinite(RN32(x_hat *
+ *     RN32(1 / RN32(s * g_x)))), the sign of a zero result kept.
+ *   INT4 (group 64; g_x ignored): s_h = fp16(RN32(amax/7)); s_h == 0 ->
+ *     codes 0; else q = clamp(rint(RN32(x_hat * RN32(1/s_h))), -8, 7).
+ *   lora_act[m,t] = sum_k X[m,k] * L1s[t,k] (fp32 accumulation), then
+ *     multiplied by RN32(1 / RN32(g_x * g_w)) (NVFP4; 1 for INT4) and
+ *     rounded to tf32 (10-bit mantissa): the unit of the GEMM accumulator.
+ * X [device] M x K bf16.  Outputs [device]: qx M x K/2 bytes; sx
+ * svdq_act_scale_bytes(w, M) bytes (padding rows are written with zeros);
+ * lora_act M x rank_pad fp32 (may be NULL when rank == 0). */
+SVDQ_API svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
+                                        uint8_t* qx, void* sx, float* lora_act, void* stream);
+
+/* 4-bit GEMM with the lora-up and the bias fused into its epilogue:
+ *   NVFP4: Y = RN32(g_x * g_w) * (sum_b s_x s_w sum_{k in b} e2m1(qx) e2m1(qw)
+ *                                 + lora_act L2^T) + b
+ *   INT4:  Y = sum_g s_x s_w sum_{k in g} qx qw + lora_act L2^T + b
+ * stored as bf16 (RNE) or fp32 (out_dtype).  Inputs as written by
+ * svdq_quantize_act_lora_down.  Y [device] M x N. */
+SVDQ_API svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
+                                   const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream);
+
+/* Workspace bytes of svdq_linear_forward for M rows (qx, sx, lora_act). */
+SVDQ_API size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M);
+
+/* The whole layer: svdq_quantize_act_lora_down then svdq_w4a4_gemm_lora_up
+ * on one stream, intermediates in `workspace` [device] (>=
+ * svdq_workspace_bytes(w, M), 1024-byte aligned). */
+SVDQ_API svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
+                                int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream` and returns (then clears) the status word that the
+ * GEMM kernels of this weight set write when a bounded wait runs out:
+ * SVDQ_ERR_TIMEOUT, else SVDQ_OK (or SVDQ_ERR_CUDA if the sync failed). */
+SVDQ_API svdq_status svdq_device_status(const svdq_weights* w, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */
