@@ -259,7 +259,7 @@ def test_argument_errors(svdq):
         svdq.svdq_linear_forward(w, X, M, 0.0, Y, ws, ws.numel())
     assert e.value.status == 1
     with pytest.raises(svdq.SVDQError) as e:
-        svdq.svdq_linear_forward(w, X, M, float(ol.gx), Y.view(torch.uint8)[1:], ws, ws.numel())
+        svdq.svdq_linear_forward(w, X, M, float(ol.gx), Y.reshape(-1).view(torch.uint8)[2:], ws, ws.numel())
     assert e.value.status == 3
     svdq.svdq_linear_forward(w, X, 0, float(ol.gx), Y, ws, ws.numel())  # M = 0 is a no-op
     bad = svdq.make_desc(100, 256, 16)
