@@ -71,6 +71,7 @@ _SIGS = {
     "svdq_w4a4_gemm_lora_up": (_I, [_P, _P, _P, _F, _P, _I, _P, _I, _P]),
     "svdq_workspace_bytes": (_Z, [_P, _I]),
     "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
+    "svdq_linear_forward_noalloc": (_I, [_P, _P, _I, _F, _P, _I, _P]),
     "svdq_device_status": (_I, [_P, _P]),
 }
 
@@ -199,6 +200,16 @@ def svdq_linear_forward(w: Weights, X, M: int, g_x: float, Y, workspace, ws_byte
                         out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
     _check(load_library().svdq_linear_forward(w.handle, _ptr(X), M, float(g_x), _ptr(Y), out_dtype, _ptr(workspace),
                                               ws_bytes, _stream(stream)), "svdq_linear_forward")
+
+
+def svdq_linear_forward_noalloc(w: Weights, X, M: int, g_x: float, Y, out_dtype: int = SVDQ_OUT_BF16,
+                                stream=None) -> None:
+    """The forward for callers that cannot allocate device memory: the
+    intermediates live in the library's own static device scratch (16 MiB;
+    larger M raises SVDQ_ERR_WORKSPACE).  Calls that overlap on the GPU race
+    on that scratch."""
+    _check(load_library().svdq_linear_forward_noalloc(w.handle, _ptr(X), M, float(g_x), _ptr(Y), out_dtype,
+                                                      _stream(stream)), "svdq_linear_forward_noalloc")
 
 
 def svdq_device_status(w: Weights, stream=None) -> int:

@@ -203,6 +203,27 @@ SVDQ_API size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M);
 SVDQ_API svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
                                 int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream);
 
+/* The layer forward without a caller-provided workspace.  No counterpart
+ * in the pages: this exists for callers that cannot allocate device memory
+ * at all, for example code that runs under a host framework which owns
+ * every device allocation through its own pool and forbids extra ones, or
+ * a latency-critical serving loop that must never call cudaMalloc (which
+ * can synchronise the device).  The intermediates (codes, scales,
+ * lora_act) live in one static device array of 16 MiB that every GPU
+ * loading this library holds until the process exits.
+ * Same computation and arguments as svdq_linear_forward minus the
+ * workspace; returns SVDQ_ERR_WORKSPACE when svdq_workspace_bytes(w, M)
+ * plus 1024 bytes of alignment exceeds 16 MiB (e.g. M = 4608 at K = 3072
+ * fits; M = 9216 does not).  Allocates nothing: no cudaMalloc, cudaFree
+ * or allocating library call.  The first call on each device looks up the
+ * array's device address (with that device current), so make that first
+ * call before any stream capture.  All calls on a device share the array
+ * and leave the last call's intermediates in it; every call rewrites all
+ * it reads, so nothing needs clearing, but calls that overlap on the GPU
+ * (other streams, other host threads) race on it. */
+SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
+                                                 void* Y, int32_t out_dtype, void* stream);
+
 /* Synchronises `stream` and returns (then clears) the status word that the
  * GEMM kernels of this weight set write when a bounded wait runs out:
  * SVDQ_ERR_TIMEOUT, else SVDQ_OK (or SVDQ_ERR_CUDA if the sync failed). */
