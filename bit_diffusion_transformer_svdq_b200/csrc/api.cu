@@ -61,7 +61,7 @@ int num_sms(int device) {
 }
 
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
-                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -75,7 +75,8 @@ bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -190,12 +191,19 @@ svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, co
   w->amax = reinterpret_cast<uint32_t*>(b + L.amax);
 
   bool ok = encode_tmap_2d(&w->tm_qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qw, desc->K / 2, desc->N, desc->K / 2, 128,
-                           256);
-  if (ok && w->rank_pad > 0)
+                           128);
+  if (ok && desc->precision == SVDQ_NVFP4)
+    ok = encode_tmap_2d(&w->tm_sw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sw, 256, L.sw_bytes / 256, 256, 256, 8, false);
+  if (ok && w->rank_pad > 0) {
     ok = encode_tmap_2d(&w->tm_l2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->l2, w->rank_pad, desc->N,
-                        static_cast<uint64_t>(w->rank_pad) * 4, 32, 256);
-  else
+                        static_cast<uint64_t>(w->rank_pad) * 4, 32, 128);
+    if (ok)
+      ok = encode_tmap_2d(&w->tm_l1s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1s, desc->K, w->rank_pad,
+                          static_cast<uint64_t>(desc->K) * 2, 64, w->rank_pad);
+  } else {
     w->tm_l2 = w->tm_qw;
+    w->tm_l1s = w->tm_qw;
+  }
   if (!ok) {
     std::free(w);
     return SVDQ_ERR_CUDA;

@@ -1,23 +1,31 @@
 // The 4-bit GEMM of the SVDQuant W4A4 layer with the lora-up and the bias
 // fused into the epilogue (charmloop.ai Nunchaku news item, second
-// paragraph: "the up-projection into the 4-bit compute kernel").
+// paragraph: the up-projection runs inside the 4-bit compute kernel).
 //
-// sm_100a design, one persistent CTA per SM, 128 x 256 output tiles:
-//   warp 0      TMA producer: qx / qw tiles (128-byte swizzle) and the
-//               per-16 E4M3 scale atoms (bulk copies) into a 4-stage ring.
-//   warp 1      TMEM owner and MMA issuer: per tile, ceil(rank/32) ring
-//               slots carry the lora_act / L2 tiles and are multiplied with
-//               tcgen05 kind::tf32 into the accumulator, then every K stage
-//               copies its scales to TMEM (tcgen05.cp) and issues
-//               tcgen05 kind::mxf4nvf4 block-scaled MMAs (K = 64 each).
-//   warps 2-9   epilogue: drain the 128 x 256 fp32 accumulator from TMEM,
-//               release it to the MMA warp, then y = acc * g_x g_w + b.
+// sm_100a design: CTA pairs (clusters of 2) run tcgen05 cta_group::2 MMAs on
+// 256 x 256 output tiles; the pair is persistent over the tile list.
+// Each CTA stages its own 128 rows of A (codes of X_hat) and its own 128
+// rows of B (codes of R) per 256-wide K step, so a pair reads the B tile
+// once for 256 output rows: 38 KB per SM per K step instead of the 54 KB of
+// a 128 x 256 single-CTA tile.  All loads are plain 2-D TMA copies into the
+// issuing CTA's own shared memory, counted on the first CTA's barrier.
+//   warp 0      TMA producer (both CTAs): codes, per-16 E4M3 scale atoms,
+//               and, per tile, the lora_act / L2 slots of the low-rank branch.
+//   warp 1      TMEM owner (both CTAs); in the first CTA the MMA issuer:
+//               tf32 lora-up MMAs into the accumulator, then per K step the
+//               scale copies to TMEM (tcgen05.cp) and the block-scaled
+//               kind::mxf4nvf4 MMAs (K = 64 each).
+//   warps 2-9   epilogue (both CTAs): drain the CTA's 128 x 256 fp32 rows
+//               from TMEM, release them to the MMA issuer, then
+//               y = acc * RN32(g_x g_w) + b, stored as bf16 or fp32.
 // The lora-up shares the accumulator with the 4-bit product because
-// lora_act arrives pre-divided by g_x g_w: one TMEM read per output.
+// lora_act arrives pre-divided by g_x g_w.
 //
-// TMEM columns: [0, 256) accumulator, [256, 272) A scales, [272, 304) B
-// scales (4 x 32-bit columns per 128 rows per MMA; lane i of every 32-lane
-// quarter holds rows i, i+32, i+64, i+96 in its four columns).
+// TMEM columns (same in both CTAs): [0, 256) accumulator (this CTA's 128
+// rows), then one scale slot of 48 columns per ring stage: 16 columns of A
+// scales (this CTA's rows) and 32 of B scales (all 256 columns; each CTA
+// holds a copy), 4 x 32-bit columns per 128 rows per MMA; lane i of every
+// 32-lane quarter holds rows i, i+32, i+64, i+96.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -28,33 +36,32 @@
 namespace svdq {
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 256;  // rows of a pair tile (128 per CTA)
 constexpr int BN = 256;
 constexpr int BK = 256;  // fp4 elements per ring stage (128 bytes per row)
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK / 2;                                   // 16 KB
-constexpr int kBBytes = BN * BK / 2;                                   // 32 KB
-constexpr int kSfaBytes = BM * BK / 16;                                // 2 KB
-constexpr int kSfbBytes = BN * BK / 16;                                // 4 KB
-constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 54 KB
+constexpr int kStages = 5;
+constexpr int kABytes = 128 * BK / 2;                                  // 16 KB
+constexpr int kBBytes = 128 * BK / 2;                                  // 16 KB (this CTA's N half)
+constexpr int kSfaBytes = 128 * BK / 16;                               // 2 KB
+constexpr int kSfbBytes = 256 * BK / 16;                               // 4 KB (all 256 N)
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc = 0, kColSfa = 256, kColSfb = 272;
+constexpr uint32_t kColAcc = 0, kColSf = 256, kSfSlotCols = 48;
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kColSf + kStages * kSfSlotCols <= kTmemCols, "TMEM budget");
 
 // Instruction descriptors (kind::mxf4nvf4 block-scaled and kind::tf32),
-// M = 128, N = 256, both operands K-major.
+// M = 256 (a CTA pair), N = 256, both operands K-major.
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 constexpr uint32_t kIdescTf32 =
     (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 
 struct GemmParams {
-  const uint8_t* sfa;
-  const uint8_t* sfb;
   const float* bias;
   void* Y;
   int* status;
@@ -65,6 +72,7 @@ struct GemmParams {
 template <bool kF32Out>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                       const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -79,11 +87,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs; 1: its peer
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
   const int num_m = (p.M + BM - 1) / BM;
   const int num_n = (p.N + BN - 1) / BN;
   const int num_tiles = num_m * num_n;
-  const int k_sub = p.K / 64;               // 64-wide MMA steps along K
-  const int num_kb = (k_sub + 3) / 4;       // ring stages per tile for the 4-bit product
+  const int k_sub = p.K / 64;           // 64-wide MMA steps along K
+  const int num_kb = (k_sub + 3) / 4;   // ring stages per tile for the 4-bit product
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -91,111 +102,119 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(acc_empty, 2 * kEpiWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-    if (p.n_lora) {
-      prefetch_tmap(&tm_la);
-      prefetch_tmap(&tm_lb);
-    }
-  }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrive or TMA completion
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   uint32_t issued_mask = 0, issued_par = 0;  // producer bookkeeping for the teardown drain
 
   if (warp == 0) {
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        const int mb = tile % num_m, nb = tile / num_m;
-        const int m0 = mb * BM, n0 = nb * BN;
-        for (int j = 0; j < p.n_lora; ++j) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
+    // ------------------------------------------------ TMA producer (whole warp)
+    if (elect_one()) {
+      prefetch_tmap(&tm_a);
+      prefetch_tmap(&tm_b);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const int mb = tile % num_m, nb = tile / num_m;
+      const int m_cta = mb * BM + 128 * static_cast<int>(rank);  // this CTA's A rows
+      const int n_cta = nb * BN + 128 * static_cast<int>(rank);  // this CTA's B rows
+      for (int j = 0; j < p.n_lora; ++j) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
+        if (elect_one()) {
           uint8_t* st = smem + stage * kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes);
-          tma_load_2d(st, &tm_la, 32 * j, m0, &full[stage]);
-          tma_load_2d(st + kABytes, &tm_lb, 32 * j, n0, &full[stage]);
-          issued_mask |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (kABytes + kBBytes));
+          tma_load_2d_pair(st, &tm_la, 32 * j, m_cta, fb);
+          tma_load_2d_pair(st + kABytes, &tm_lb, 32 * j, n_cta, fb);
         }
-        for (int kb = 0; kb < num_kb; ++kb) {
-          const int nsub = min(4, k_sub - 4 * kb);
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
+        __syncwarp();
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
+        if (elect_one()) {
           uint8_t* st = smem + stage * kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], kABytes + kBBytes + 3 * nsub * 512);
-          tma_load_2d(st, &tm_a, kb * 128, m0, &full[stage]);
-          tma_load_2d(st + kABytes, &tm_b, kb * 128, n0, &full[stage]);
-          const size_t sf_off = static_cast<size_t>(4 * kb) * 512;
-          bulk_load(st + kABytes + kBBytes, p.sfa + static_cast<size_t>(mb) * k_sub * 512 + sf_off, nsub * 512,
-                    &full[stage]);
-          bulk_load(st + kABytes + kBBytes + kSfaBytes, p.sfb + static_cast<size_t>(2 * nb) * k_sub * 512 + sf_off,
-                    nsub * 512, &full[stage]);
-          bulk_load(st + kABytes + kBBytes + kSfaBytes + 2048,
-                    p.sfb + static_cast<size_t>(2 * nb + 1) * k_sub * 512 + sf_off, nsub * 512, &full[stage]);
-          issued_mask |= 1u << stage;
-          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * kStageBytes);
+          tma_load_2d_pair(st, &tm_a, kb * 128, m_cta, fb);
+          tma_load_2d_pair(st + kABytes, &tm_b, kb * 128, n_cta, fb);
+          // scale atoms: rows of 256 bytes, 8 rows = the 4 atoms of this K step
+          tma_load_2d_pair(st + kABytes + kBBytes, &tm_sfa, 0, ((m_cta >> 7) * k_sub + 4 * kb) * 2, fb);
+          tma_load_2d_pair(st + kABytes + kBBytes + kSfaBytes, &tm_sfb, 0, ((nb * 2) * k_sub + 4 * kb) * 2, fb);
+          tma_load_2d_pair(st + kABytes + kBBytes + kSfaBytes + 2048, &tm_sfb, 0,
+                           ((nb * 2 + 1) * k_sub + 4 * kb) * 2, fb);
         }
+        __syncwarp();
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    // ----------------------------------- MMA issuer (whole warp, first CTA only)
+    if (rank == 0) {
       int stage = 0;
       uint32_t phase = 0, acc_phase = 0;
       const uint32_t d_acc = tmem + kColAcc;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(acc_empty, acc_phase ^ 1, abort_flag)) goto teardown;
+      for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+        if (!mbar_wait_warp(acc_empty, acc_phase ^ 1, abort_flag)) goto teardown;
         tc_fence_after();
         uint32_t accumulate = 0;
         for (int j = 0; j < p.n_lora; ++j) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto teardown;
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-          const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kABytes);
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+            const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kABytes);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {  // 4 x K=8 tf32 steps of 32 bytes
-            mma_tf32(d_acc, da + 2 * k, db + 2 * k, kIdescTf32, accumulate);
-            accumulate = 1;
+            for (int k = 0; k < 4; ++k)  // 4 x K=8 tf32 steps of 32 bytes
+              mma_tf32_pair(d_acc, da + 2 * k, db + 2 * k, kIdescTf32, (accumulate | k) ? 1u : 0u);
+            tc_commit_pair(&empty[stage], 0x3);
           }
-          tc_commit(&empty[stage]);
+          __syncwarp();
+          accumulate = 1;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
         for (int kb = 0; kb < num_kb; ++kb) {
           const int nsub = min(4, k_sub - 4 * kb);
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto teardown;
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-          const uint32_t s_sfa = sa + kABytes + kBBytes;
-          const uint32_t s_sfb = s_sfa + kSfaBytes;
-          for (int k = 0; k < nsub; ++k) {
-            tc_cp_32x128b_warpx4(tmem + kColSfa + 4 * k, sdesc_rows16(s_sfa + 512 * k));
-            tc_cp_32x128b_warpx4(tmem + kColSfb + 8 * k, sdesc_rows16(s_sfb + 512 * k));
-            tc_cp_32x128b_warpx4(tmem + kColSfb + 8 * k + 4, sdesc_rows16(s_sfb + 2048 + 512 * k));
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+            const uint32_t s_sfa = sa + kABytes + kBBytes;
+            const uint32_t s_sfb = s_sfa + kSfaBytes;
+            const uint32_t t_sfa = tmem + kColSf + stage * kSfSlotCols;
+            const uint32_t t_sfb = t_sfa + 16;
+            const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kABytes);
+            // scale copies and MMAs alternate so that each copy overlaps the
+            // MMA issued just before it in the tensor pipe's in-order stream
+            for (int k = 0; k < nsub; ++k) {  // K=64 fp4 steps of 32 bytes
+              tc_cp_32x128b_warpx4_pair(t_sfa + 4 * k, sdesc_rows16(s_sfa + 512 * k));
+              tc_cp_32x128b_warpx4_pair(t_sfb + 8 * k, sdesc_rows16(s_sfb + 512 * k));
+              tc_cp_32x128b_warpx4_pair(t_sfb + 8 * k + 4, sdesc_rows16(s_sfb + 2048 + 512 * k));
+              mma_nvfp4_pair(d_acc, da + 2 * k, db + 2 * k, kIdescNvfp4, t_sfa + 4 * k, t_sfb + 8 * k,
+                             (accumulate | k) ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[stage], 0x3);
           }
-          const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kABytes);
-          for (int k = 0; k < nsub; ++k) {  // K=64 fp4 steps of 32 bytes
-            mma_nvfp4(d_acc, da + 2 * k, db + 2 * k, kIdescNvfp4, tmem + kColSfa + 4 * k, tmem + kColSfb + 8 * k,
-                      accumulate);
-            accumulate = 1;
-          }
-          tc_commit(&empty[stage]);
+          __syncwarp();
+          accumulate = 1;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        tc_commit(acc_full);
+        if (elect_one()) tc_commit_pair(acc_full, 0x3);
+        __syncwarp();
         acc_phase ^= 1;
       }
     }
@@ -203,9 +222,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------- epilogue
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
+    const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int m0 = (tile % num_m) * BM, n0 = (tile / num_m) * BN;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+      const int m0 = (tile % num_m) * BM + 128 * static_cast<int>(rank), n0 = (tile / num_m) * BN;
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
       acc_phase ^= 1;
       tc_fence_after();
@@ -216,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acc_empty);
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
       const int row = m0 + quarter * 32 + lane;
       if (row < p.M) {
@@ -254,20 +274,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 teardown:
   __syncthreads();
-  if (warp == 0 && lane == 0) {
-    // every TMA / bulk copy this CTA issued must land before shared memory is released
+  if (rank == 0 && warp == 0 && lane == 0) {
+    // every TMA copy of the pair completes on the first CTA's barriers:
+    // they must all have landed before either CTA releases its memory
     for (int s = 0; s < kStages; ++s)
       if (issued_mask & (1u << s)) mbar_wait_limited(&full[s], (issued_par >> s) & 1u, 200000000ull);
   }
-  if (warp == 1 && lane == 0) {
-    tc_commit(drain);  // arrives once every MMA / copy issued so far has finished
-    mbar_wait_limited(drain, 0, 200000000ull);
+  if (rank == 0 && warp == 1) {
+    // the lane that issued the MMAs commits: arrives once all of them have finished
+    if (elect_one()) {
+      tc_commit_pair(drain, 0x1);
+      mbar_wait_limited(drain, 0, 200000000ull);
+    }
+    __syncwarp();
   }
   if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, static_cast<int>(SVDQ_ERR_TIMEOUT));
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 1) tmem_dealloc_pair(tmem, kTmemCols);
 }
 
 }  // namespace
@@ -275,19 +300,21 @@ teardown:
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
                               const float* lora_act, int M, void* Y, int out_dtype, cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N;
-  CUtensorMap tm_a, tm_la;
-  if (!encode_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K / 2, M, K / 2, 128, BM))
+  const int64_t m_pad = m_pad_of(M);
+  CUtensorMap tm_a, tm_sfa, tm_la;
+  if (!encode_tmap_2d(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K / 2, M, K / 2, 128, 128))
+    return cudaErrorInvalidValue;
+  if (!encode_tmap_2d(&tm_sfa, CU_TENSOR_MAP_DATA_TYPE_UINT8, sx, 256, nvfp4_scale_bytes(m_pad, K) / 256, 256, 256, 8,
+                      false))
     return cudaErrorInvalidValue;
   if (w->rank_pad > 0) {
     if (!encode_tmap_2d(&tm_la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lora_act, w->rank_pad, M,
-                         static_cast<uint64_t>(w->rank_pad) * 4, 32, BM))
+                        static_cast<uint64_t>(w->rank_pad) * 4, 32, 128))
       return cudaErrorInvalidValue;
   } else {
     tm_la = tm_a;  // unused when there is no low-rank branch
   }
   GemmParams p;
-  p.sfa = sx;
-  p.sfb = static_cast<const uint8_t*>(w->sw);
   p.bias = w->bias;
   p.Y = Y;
   p.status = w->status;
@@ -297,12 +324,23 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   p.n_lora = w->rank_pad / 32;
   p.gxgw = g_x * w->g_w;  // RN32(g_x * g_w)
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = std::min(tiles, num_sms(w->device));
+  const int pairs = std::min(tiles, num_sms(w->device) / 2);
   auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, s>>>(tm_a, w->tm_qw, tm_la, w->tm_l2, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_a, w->tm_qw, tm_sfa, w->tm_sw, tm_la, w->tm_l2, p);
 }
 
 }  // namespace svdq

@@ -46,11 +46,13 @@ struct svdq_weights {
   float* l2;
   float* inv_lambda;
   float* bias;
-  int* status;    // written by GEMM kernels when a bounded wait runs out
+  int* status;    // written by the kernels when a bounded wait runs out
   uint32_t* amax; // scratch word of the preparation pass
   int device;
-  CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes
-  CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes
+  CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
+  CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows
+  CUtensorMap tm_sw;  // NVFP4 weight scales viewed as rows of 256 bytes, boxes of 8 rows (4 atoms)
+  CUtensorMap tm_l1s; // bf16 L1s, 64-column 128-byte swizzled boxes of all rank_pad rows
 };
 
 namespace svdq {
@@ -72,7 +74,7 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
 // link-time dependency on libcuda).  2-D, row-major, `inner` elements per
 // row of `row_bytes` stride, box {box_inner, box_rows}, 128-byte swizzle.
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
-                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows);
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128 = true);
 
 int num_sms(int device);
 

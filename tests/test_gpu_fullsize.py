@@ -1,0 +1,63 @@
+"""Parity at the full workload sizes, in the launch configuration the bench
+uses: every weight and activation code and scale bit-exact against the
+oracle; Y checked on seeded sampled rows (rows are independent given the
+codes, so the oracle computes only those rows)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import svdq as V
+from tests import svdq_testlib as T
+
+pytestmark = pytest.mark.gpu
+
+REL_F = 2e-3
+MAX_ABS = 1e-2
+SAMPLE_ROWS = 96
+
+
+@pytest.fixture(scope="module")
+def svdq():
+    if not torch.cuda.is_available():
+        pytest.fail("no CUDA device")
+    from bit_diffusion_transformer_svdq_b200 import svdq as mod
+    mod.load_library()
+    return mod
+
+
+@pytest.mark.parametrize("workload", ["qkv", "mlp_up", "mlp_down"])
+def test_full_size_nvfp4(svdq, workload):
+    li = synth.make_layer(workload, 2)
+    M, K, N = li.shape.M, li.shape.K, li.shape.N
+    ol = T.oracle_layer(li)
+    w = T.gpu_prepare(svdq, li, ol)
+    h = T.weights_to_host(w)
+    assert h["g_w"] == ol.prep.g_w
+    assert np.array_equal(T.unpack_codes(h["qw"]), ol.prep.qw)
+    assert np.array_equal(T.untile_nvfp4_scales(h["sw"], N, K), ol.prep.sw)
+
+    X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
+    rows = np.sort(np.random.default_rng(7).choice(M, SAMPLE_ROWS, replace=False))
+    xs = li.x[rows]
+    act = V.quantize_activations(xs, ol.prep, ol.gx)
+    codes = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
+    assert np.array_equal(codes[rows], act.qx)
+    assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K)[rows], act.sx)
+
+    ref = V.forward_from_codes(act, ol.prep, ol.gx)
+    rms = np.sqrt(np.mean(ref ** 2))
+    for out_dtype in (1, 0):
+        Y = torch.empty((M, N), dtype=torch.float32 if out_dtype else torch.bfloat16, device="cuda")
+        svdq.svdq_w4a4_gemm_lora_up(w, qx, sx, float(ol.gx), la, M, Y, out_dtype)
+        torch.cuda.synchronize()
+        y = Y.float().cpu().numpy()[rows].astype(np.float64)
+        d = y - ref
+        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F
+        if out_dtype:
+            assert np.abs(d).max() <= MAX_ABS * rms
+        else:
+            half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
+            assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
+        assert np.all(np.isfinite(Y.float().cpu().numpy()))
+    assert svdq.svdq_device_status(w) == 0
