@@ -81,6 +81,21 @@ bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_chunked_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows,
+                              uint32_t box_chunks) {
+  CUtensorMap probe;
+  if (!encode_tmap_2d(&probe, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, K, rows, K * 2, 64, box_rows))
+    return false;  // also loads the encoder entry point
+  cuuint64_t dims[3] = {64, rows, K / 64};
+  cuuint64_t strides[2] = {K * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, box_chunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 WeightLayout weight_layout(const svdq_layer_desc& d) {
   WeightLayout L{};
   const int rp = rank_pad_of(d.rank);
@@ -198,8 +213,7 @@ svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, co
     ok = encode_tmap_2d(&w->tm_l2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->l2, w->rank_pad, desc->N,
                         static_cast<uint64_t>(w->rank_pad) * 4, 32, 128);
     if (ok)
-      ok = encode_tmap_2d(&w->tm_l1s, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1s, desc->K, w->rank_pad,
-                          static_cast<uint64_t>(desc->K) * 2, 64, w->rank_pad);
+      ok = encode_tmap_chunked_bf16(&w->tm_l1s, w->l1s, w->rank_pad, desc->K, w->rank_pad, kQChunks);
   } else {
     w->tm_l2 = w->tm_qw;
     w->tm_l1s = w->tm_qw;

@@ -52,7 +52,7 @@ struct svdq_weights {
   CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_sw;  // NVFP4 weight scales viewed as rows of 256 bytes, boxes of 8 rows (4 atoms)
-  CUtensorMap tm_l1s; // bf16 L1s, 64-column 128-byte swizzled boxes of all rank_pad rows
+  CUtensorMap tm_l1s; // bf16 L1s as 64-column chunks: boxes of all rank_pad rows x kQChunks chunks
 };
 
 namespace svdq {
@@ -75,6 +75,16 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
 // row of `row_bytes` stride, box {box_inner, box_rows}, 128-byte swizzle.
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128 = true);
+// A K-major bf16 matrix (rows x K, row pitch K * 2 bytes) seen as 64-column
+// chunks: dims {64, rows, K / 64}.  A {64, box_rows, box_chunks} box lands
+// in shared memory as box_chunks consecutive 128-byte-swizzled tiles of
+// box_rows x 64, the same bytes that box_chunks separate 2-D boxes would
+// write, in one request.
+bool encode_tmap_chunked_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows,
+                              uint32_t box_chunks);
+
+// 64-column chunks per stage of the activation quantiser (the L1s map's box).
+constexpr int kQChunks = 1;
 
 int num_sms(int device);
 

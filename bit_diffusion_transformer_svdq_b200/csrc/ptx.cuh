@@ -83,6 +83,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int32_t
       : "memory");
 }
 
+// 3-D tiled load (same completion rule as the 2-D form).
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, int32_t x, int32_t y, int32_t z,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -269,7 +279,7 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
 // element 0 in bits 0..3.
 __device__ __forceinline__ uint32_t pack8_e2m1(const float* v) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
@@ -344,7 +354,7 @@ __device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64
 // Two fp32 -> two E2M1 (RNE, satfinite) in one byte, `lo` in bits 0..3.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 b0;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
       "cvt.u32.u8 %0, b0;\n\t}\n"
@@ -356,7 +366,7 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 // fp32 -> E4M3 (RNE, satfinite), in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(v), "f"(0.0f));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(v), "f"(0.0f));
   return static_cast<uint32_t>(out) & 0xFFu;
 }
 
@@ -364,14 +374,14 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   uint16_t in = static_cast<uint16_t>(code & 0xFFu);
   uint32_t h2;
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 
 // fp32 -> tf32 bit pattern (round to nearest, ties away from zero).
 __device__ __forceinline__ float round_tf32(float v) {
   uint32_t out;
-  asm volatile("cvt.rna.tf32.f32 %0, %1;" : "=r"(out) : "f"(v));
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(out) : "f"(v));
   return __uint_as_float(out);
 }
 
