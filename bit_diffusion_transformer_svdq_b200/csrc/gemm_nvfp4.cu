@@ -17,7 +17,9 @@
 //               kind::mxf4nvf4 MMAs (K = 64 each).
 //   warps 2-9   epilogue (both CTAs): drain the CTA's 128 x 256 fp32 rows
 //               from TMEM, release them to the MMA issuer, then
-//               y = acc * RN32(g_x g_w) + b, stored as bf16 or fp32.
+//               y = acc * RN32(g_x g_w) + b (the tile's bias read once into
+//               shared memory), written as bf16 or fp32 into 128-byte-
+//               swizzled staging boxes and stored by TMA in whole lines.
 // The lora-up shares the accumulator with the 4-bit product because
 // lora_act arrives pre-divided by g_x g_w.
 //
@@ -39,7 +41,7 @@ namespace {
 constexpr int BM = 256;  // rows of a pair tile (128 per CTA)
 constexpr int BN = 256;
 constexpr int BK = 256;  // fp4 elements per ring stage (128 bytes per row)
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kABytes = 128 * BK / 2;                                  // 16 KB
 constexpr int kBBytes = 128 * BK / 2;                                  // 16 KB (this CTA's N half)
 constexpr int kSfaBytes = 128 * BK / 16;                               // 2 KB
@@ -49,7 +51,11 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0, kColSf = 256, kSfSlotCols = 48;
-constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int kStagingPerWarp = 8192;  // two 32-row x 128-byte output boxes per epilogue warp
+constexpr int kStagingOff = kStages * kStageBytes;
+constexpr int kBiasOff = kStagingOff + kEpiWarps * kStagingPerWarp;  // 2 x 256 floats
+constexpr int kBarOff = kBiasOff + 2 * BN * 4;
+constexpr size_t kSmemBytes = kBarOff + 256 /*barriers*/ + 1024 /*align*/;
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -67,6 +73,7 @@ struct GemmParams {
   int* status;
   int M, N, K, n_lora;
   float gxgw;
+  int tma_store;  // Y rows are whole multiples of 16 bytes: store through tm_y
 };
 
 template <bool kF32Out>
@@ -74,10 +81,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
-                      const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * kStageBytes);
+  float* bias_s = reinterpret_cast<float*>(smem + kBiasOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
@@ -220,57 +228,94 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
+    // Warp (quarter, half) owns rows quarter*32 .. +31 (its TMEM lane
+    // quarter) and columns half*128 .. +127 of the CTA's 128 x 256 tile.
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
+    const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue warps
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+    uint8_t* const stg = smem + kStagingOff + (warp - 2) * kStagingPerWarp;  // 128-byte-swizzled boxes
     uint32_t acc_phase = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs) {
+    int tcount = 0;
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
       const int m0 = (tile % num_m) * BM + 128 * static_cast<int>(rank), n0 = (tile / num_m) * BN;
+      // the tile's 256 bias values, once, into this tile's half of the double buffer
+      float* bias_t = bias_s + (tcount & 1) * BN;
+      bias_t[et] = n0 + et < p.N ? __ldg(p.bias + n0 + et) : 0.0f;
+      named_bar_sync(1, 32 * kEpiWarps);
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
       acc_phase ^= 1;
       tc_fence_after();
-      uint32_t v[4][32];
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColAcc + half * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(taddr + 32 * c, v[c]);
+      uint32_t v[128];  // this warp's 32 rows x 128 columns, one load
+      tmem_ld128(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColAcc + half * 128, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // the accumulator is free for the next tile
 
       const int row = m0 + quarter * 32 + lane;
-      if (row < p.M) {
+      const float* bb = bias_t + half * 128;
+      if (p.tma_store) {
+        // y rows into 128-byte-wide swizzled boxes (32 rows each), then TMA
+        // stores of whole lines; rows past M / columns past N are clipped
+        constexpr int kColsPerBox = kF32Out ? 32 : 64;
+        constexpr int kPasses = kF32Out ? 2 : 1;  // 64 or 128 columns per staging fill
+#pragma unroll
+        for (int pass = 0; pass < kPasses; ++pass) {
+          if (lane == 0) bulk_wait_read_all();  // the previous stores no longer read the boxes
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 128 / kPasses; j += 4) {
+            const int col = pass * (128 / kPasses) + j;  // within the warp's 128 columns
+            const uint32_t* a = &v[col];
+            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(a[0]), p.gxgw), bb[col]);
+            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(a[1]), p.gxgw), bb[col + 1]);
+            const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(a[2]), p.gxgw), bb[col + 2]);
+            const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(a[3]), p.gxgw), bb[col + 3]);
+            const int lc = col - pass * (128 / kPasses);   // column within this fill
+            const int box = lc / kColsPerBox;
+            const int byte = (lc % kColsPerBox) * (kF32Out ? 4 : 2);  // within the box's 128-byte row
+            uint8_t* line = stg + box * 4096 + lane * 128;
+            if constexpr (kF32Out) {
+              *reinterpret_cast<float4*>(line + (((byte >> 4) ^ (lane & 7)) << 4)) = make_float4(y0, y1, y2, y3);
+            } else {
+              __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1), h1 = __floats2bfloat162_rn(y2, y3);
+              *reinterpret_cast<uint2*>(line + (((byte >> 4) ^ (lane & 7)) << 4) + (byte & 15)) =
+                  make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < 128 / kPasses / kColsPerBox; ++b)
+              tma_store_2d(&tm_y, stg + b * 4096, n0 + half * 128 + pass * (128 / kPasses) + b * kColsPerBox,
+                           m0 + quarter * 32);
+            bulk_commit_group();
+          }
+        }
+      } else if (row < p.M) {
+        // rows whose byte length is not a multiple of 16: plain stores
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            const int n = n0 + half * 128 + 32 * c + i;
+          for (int i = 0; i < 32; ++i) {
+            const int col = 32 * c + i;
+            const int n = n0 + half * 128 + col;
             if (n < p.N) {
-              const float4 b0 = __ldg(reinterpret_cast<const float4*>(p.bias + n));
-              const float4 b1 = __ldg(reinterpret_cast<const float4*>(p.bias + n + 4));
-              const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-              float y[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = __fadd_rn(__fmul_rn(__uint_as_float(v[c][i + e]), p.gxgw), bb[e]);
-              if constexpr (kF32Out) {
-                float* dst = static_cast<float*>(p.Y) + static_cast<size_t>(row) * p.N + n;
-                reinterpret_cast<float4*>(dst)[0] = make_float4(y[0], y[1], y[2], y[3]);
-                reinterpret_cast<float4*>(dst)[1] = make_float4(y[4], y[5], y[6], y[7]);
-              } else {
-                uint4 o;
-                __nv_bfloat162 h;
-                h = __floats2bfloat162_rn(y[0], y[1]); o.x = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(y[2], y[3]); o.y = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(y[4], y[5]); o.z = *reinterpret_cast<uint32_t*>(&h);
-                h = __floats2bfloat162_rn(y[6], y[7]); o.w = *reinterpret_cast<uint32_t*>(&h);
-                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + static_cast<size_t>(row) * p.N + n) = o;
-              }
+              const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
+              if constexpr (kF32Out)
+                static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
+              else
+                static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n] = __float2bfloat16_rn(y);
             }
           }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // every store of this warp has landed
   }
+
 
 teardown:
   __syncthreads();
@@ -323,6 +368,13 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   p.K = K;
   p.n_lora = w->rank_pad / 32;
   p.gxgw = g_x * w->g_w;  // RN32(g_x * g_w)
+  // Y through TMA stores when its rows are whole multiples of 16 bytes
+  const bool f32 = out_dtype == SVDQ_OUT_F32;
+  const uint64_t row_bytes = static_cast<uint64_t>(N) * (f32 ? 4 : 2);
+  CUtensorMap tm_y = tm_a;
+  p.tma_store = row_bytes % 16 == 0 &&
+                encode_tmap_2d(&tm_y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M,
+                               row_bytes, f32 ? 32 : 64, 32);
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int pairs = std::min(tiles, num_sms(w->device) / 2);
   auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
@@ -340,7 +392,7 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_a, w->tm_qw, tm_sfa, w->tm_sw, tm_la, w->tm_l2, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_a, w->tm_qw, tm_sfa, w->tm_sw, tm_la, w->tm_l2, tm_y, p);
 }
 
 }  // namespace svdq
