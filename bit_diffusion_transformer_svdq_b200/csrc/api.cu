@@ -60,8 +60,9 @@ int num_sms(int device) {
   return g_sms[device];
 }
 
-bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
-                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+bool encode_tmap_2d_swizzle(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                            uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                            CUtensorMapSwizzle swizzle) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -75,10 +76,15 @@ bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   const CUresult r = g_encode(tm, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128) {
+  return encode_tmap_2d_swizzle(tm, dtype, base, inner, rows, row_bytes, box_inner, box_rows,
+                                swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 bool encode_tmap_chunked_bf16(CUtensorMap* tm, const void* base, uint64_t rows, uint64_t K, uint32_t box_rows,
@@ -115,6 +121,10 @@ WeightLayout weight_layout(const svdq_layer_desc& d) {
   L.bias = take(static_cast<size_t>(d.N) * 4);
   L.status = take(16);
   L.amax = take(16);
+  if (d.precision == SVDQ_INT4) {
+    L.qw8 = take(static_cast<size_t>(np) * d.K);
+    L.swp = take(static_cast<size_t>(d.K / 64) * np * 8);
+  }
   L.total = off;
   return L;
 }
@@ -204,11 +214,17 @@ svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, co
   w->bias = reinterpret_cast<float*>(b + L.bias);
   w->status = reinterpret_cast<int*>(b + L.status);
   w->amax = reinterpret_cast<uint32_t*>(b + L.amax);
+  w->qw8 = desc->precision == SVDQ_INT4 ? reinterpret_cast<int8_t*>(b + L.qw8) : nullptr;
+  w->swp = desc->precision == SVDQ_INT4 ? reinterpret_cast<float2*>(b + L.swp) : nullptr;
 
   bool ok = encode_tmap_2d(&w->tm_qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qw, desc->K / 2, desc->N, desc->K / 2, 128,
                            128);
   if (ok && desc->precision == SVDQ_NVFP4)
     ok = encode_tmap_2d(&w->tm_sw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sw, 256, L.sw_bytes / 256, 256, 256, 8, false);
+  if (ok && desc->precision == SVDQ_INT4)
+    ok = encode_tmap_2d(&w->tm_qw8, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qw8, desc->K, w->n_pad, desc->K, 128, 128);
+  else
+    w->tm_qw8 = w->tm_qw;
   if (ok && w->rank_pad > 0) {
     ok = encode_tmap_2d(&w->tm_l2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->l2, w->rank_pad, desc->N,
                         static_cast<uint64_t>(w->rank_pad) * 4, 32, 128);

@@ -1,11 +1,375 @@
-// INT4 (group 64) variant of the 4-bit GEMM; see launch_gemm_int4.
+// INT4 (group 64) variant of the 4-bit GEMM with the low-rank up-projection
+// fused in: Y = sum_g s_x[m,g] s_w[n,g] (sum_{k in g} qx qw) + lora_act L2^T + b.
+// The 4-bit codes are unpacked to 8 bits and multiplied with tcgen05
+// kind::i8 MMAs (int32 accumulate); the scales change with every 64-group,
+// so each group's integer product leaves TMEM and is scaled into an fp32
+// accumulator held in registers.
+//
+// sm_100a design, one CTA per 128 x 128 output tile (persistent over the
+// tile list):
+//   warp 0      TMA producer: per ring stage (128 K = two groups) the packed
+//               activation codes (128 rows x 64 B, 64-byte swizzled) and the
+//               prepared int8 weight codes (128 rows x 128 B, 128-byte
+//               swizzled); per tile one stage of lora_act / L2 (fp32).
+//   warps 2-5   converters: one row each, unpack the packed activation codes
+//               into int8 in the 128-byte-swizzled layout of the MMA operand
+//               (same K permutation as the prepared weights).
+//   warp 1      TMEM owner and MMA issuer: per group two kind::i8 MMAs
+//               (K = 32) into one of two int32 accumulators (128 columns
+//               each), so a group's MMAs overlap the previous group's
+//               scaling; per tile four kind::tf32 MMAs of the lora-up into
+//               the next accumulator, as one more "group" of scale 1.
+//   warps 6-13  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM lane
+//               quarter) and 64 columns; per group it reads the int32
+//               product and adds RN(P s_w) s_x to its fp32 accumulator.
+//               RN(P s_w) is one FMA on the bit pattern magic + P (exact for
+//               |P| < 2^22; a group's |P| is at most 64 * 8 * 8), no
+//               int-to-float conversion.  Finally y = acc + b is stored.
+// The group rescale is CUDA-core work on every output element (three
+// operations per element per 64 K, against 64 MACs on the tensor core), so
+// this kernel is bound by it, not by the MMAs.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace svdq {
+namespace {
 
-cudaError_t launch_gemm_int4(const svdq_weights*, const uint8_t*, const void*, const float*, int, void*, int,
-                             cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int kTileM = 128, kTileN = 128;
+constexpr int kI4Stages = 5;
+constexpr int kApBytes = kTileM * 64;    // packed activation codes of a stage: 128 K per row
+constexpr int kA8Bytes = kTileM * 128;   // unpacked
+constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes
+constexpr int kI4StageBytes = kApBytes + kA8Bytes + kB8Bytes;  // 40 KB
+constexpr int kConvWarps = 4;
+constexpr int kI4EpiWarps = 8;
+constexpr int kI4Threads = 32 * (2 + kConvWarps + kI4EpiWarps);
+constexpr uint32_t kI4TmemCols = 256;  // two accumulators of 128 columns
+constexpr size_t kI4Smem = kI4Stages * kI4StageBytes + 1024 /*align*/ + 512 /*barriers*/;
+static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+static_assert(kI4Smem <= 232448, "shared memory budget");
+
+// kind::i8: int32 D, signed 8-bit A and B, K-major, N = 128, M = 128.
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
+// kind::tf32: fp32 D, tf32 A and B, K-major, N = 128, M = 128.
+constexpr uint32_t kIdescTf32x = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
+
+// 64-byte-swizzle descriptor-free read of the packed codes: row r, 16-byte
+// unit j lives at r * 64 + ((j ^ ((r >> 1) & 3)) << 4).
+__device__ __forceinline__ uint32_t unpack_lo(uint32_t w) {
+  return (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+}
+__device__ __forceinline__ uint32_t unpack_hi(uint32_t w) { return unpack_lo(w >> 4); }
+
+struct I4Params {
+  const __half* sx;   // [K/64][m_pad]
+  const float2* swp;  // [K/64][n_pad]
+  const float* bias;
+  void* Y;
+  int* status;
+  int M, N, K, m_pad, n_lora;
+  int64_t n_pad;
+};
+
+template <bool kF32Out>
+__global__ void __launch_bounds__(kI4Threads, 1)
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_b8,
+                     const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
+                     const I4Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4Stages * kI4StageBytes);
+  uint64_t* conv = full + kI4Stages;      // activation codes unpacked (4 converter warps)
+  uint64_t* empty = conv + kI4Stages;     // MMAs done with the stage
+  uint64_t* acc_full = empty + kI4Stages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2], 8 epilogue warps
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_m = (p.M + kTileM - 1) / kTileM;
+  const int num_n = (p.N + kTileN - 1) / kTileN;
+  const int num_tiles = num_m * num_n;
+  const int groups = p.K / 64;
+  const int num_kb = (groups + 1) / 2;  // ring stages per tile (the last may hold one group)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kI4Stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&conv[s], kConvWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kI4EpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kI4TmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  uint32_t issued_mask = 0, issued_par = 0;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (whole warp)
+    if (elect_one()) {
+      prefetch_tmap(&tm_ap);
+      prefetch_tmap(&tm_b8);
+    }
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
+      for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
+        if (elect_one()) {
+          uint8_t* st = smem + stage * kI4StageBytes;
+          if (kb < num_kb) {  // packed activation codes, prepared weight codes
+            mbar_arrive_expect_tx(&full[stage], kApBytes + kB8Bytes);
+            tma_load_2d(st, &tm_ap, kb * 64, m0, &full[stage]);
+            tma_load_2d(st + kApBytes + kA8Bytes, &tm_b8, kb * 128, n0, &full[stage]);
+          } else {  // lora_act and L2 columns 32 j .. 32 j + 31 (fp32)
+            const int j = kb - num_kb;
+            mbar_arrive_expect_tx(&full[stage], kA8Bytes + kB8Bytes);
+            tma_load_2d(st + kApBytes, &tm_la, 32 * j, m0, &full[stage]);
+            tma_load_2d(st + kApBytes + kA8Bytes, &tm_lb, 32 * j, n0, &full[stage]);
+          }
+        }
+        __syncwarp();
+        issued_mask |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp >= 2 && warp < 2 + kConvWarps) {
+    // ------------------------------------------------------- converters
+    const int r = (warp - 2) * 32 + lane;  // row of the tile
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
+        if (kb < num_kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) goto teardown;
+          const uint8_t* ap = smem + stage * kI4StageBytes + r * 64;
+          uint8_t* a8 = smem + stage * kI4StageBytes + kApBytes + r * 128;
+          uint4 in[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) in[j] = *reinterpret_cast<const uint4*>(ap + ((j ^ ((r >> 1) & 3)) << 4));
+          const uint32_t w[16] = {in[0].x, in[0].y, in[0].z, in[0].w, in[1].x, in[1].y, in[1].z, in[1].w,
+                                  in[2].x, in[2].y, in[2].z, in[2].w, in[3].x, in[3].y, in[3].z, in[3].w};
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) =
+                make_uint4(unpack_lo(w[2 * u]), unpack_hi(w[2 * u]), unpack_lo(w[2 * u + 1]), unpack_hi(w[2 * u + 1]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&conv[stage]);
+        }
+        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1) {
+    // --------------------------------------------- MMA issuer (whole warp)
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t gcount = 0;  // accumulator uses so far: buffer gcount & 1, its use gcount >> 1
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < num_kb; ++kb) {
+        if (!mbar_wait_warp(&conv[stage], phase, abort_flag)) goto teardown;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * kI4StageBytes + kApBytes);
+        const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
+        const int ng = min(2, groups - 2 * kb);
+        for (int gi = 0; gi < ng; ++gi, ++gcount) {
+          const uint32_t buf = gcount & 1;
+          if (!mbar_wait_warp(&acc_empty[buf], ((gcount >> 1) & 1) ^ 1, abort_flag)) goto teardown;
+          tc_fence_after();
+          if (elect_one()) {
+#pragma unroll
+            for (int k = 0; k < 2; ++k)  // K = 32 int8 (32 bytes) per MMA
+              mma_i8(tmem + buf * kTileN, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescI8, k ? 1u : 0u);
+            tc_commit(&acc_full[buf]);
+          }
+          __syncwarp();
+        }
+        if (elect_one()) tc_commit(&empty[stage]);
+        __syncwarp();
+        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+      }
+      if (p.n_lora > 0) {  // the lora-up as one more accumulator use, of scale 1
+        const uint32_t buf = gcount & 1;
+        if (!mbar_wait_warp(&acc_empty[buf], ((gcount >> 1) & 1) ^ 1, abort_flag)) goto teardown;
+        for (int j = 0; j < p.n_lora; ++j) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t sa = smem_u32(smem + stage * kI4StageBytes + kApBytes);
+            const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
+              mma_tf32(tmem + buf * kTileN, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
+            tc_commit(&empty[stage]);
+          }
+          __syncwarp();
+          if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+        }
+        if (elect_one()) tc_commit(&acc_full[buf]);
+        __syncwarp();
+        ++gcount;
+      }
+    }
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int q4 = warp & 3;                     // TMEM lane quarter: rows 32 q4 .. + 31
+    const int ch = (warp - 2 - kConvWarps) >> 2;  // columns 64 ch .. + 63
+    const int r = 32 * q4 + lane;
+    uint32_t gcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
+      const int row = m0 + r;
+      float acc[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+      for (int g = 0; g < groups + (p.n_lora > 0 ? 1 : 0); ++g, ++gcount) {
+        const uint32_t buf = gcount & 1;
+        if (!mbar_wait(&acc_full[buf], (gcount >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const bool lora = g == groups;
+        const float sxr = lora ? 1.0f : __half2float(p.sx[static_cast<size_t>(g) * p.m_pad + row]);
+        const float4* swq = reinterpret_cast<const float4*>(p.swp + static_cast<size_t>(lora ? 0 : g) * p.n_pad + n0 + 64 * ch);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time
+          uint32_t P[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + buf * kTileN + 64 * ch + 32 * hh, P);
+          tmem_ld_wait();
+          if (hh == 1) {  // both halves are in registers: the accumulator is free
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          }
+          if (!lora) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float4 t = __ldg(swq + (32 * hh + c) / 2);  // (s_w, -magic s_w) of two columns
+              // RN(P s_w) exactly: bits(magic) + P is the float magic + P
+              const float u0 = __fmaf_rn(__int_as_float(static_cast<int>(P[c]) + 0x4B400000), t.x, t.y);
+              const float u1 = __fmaf_rn(__int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000), t.z, t.w);
+              acc[32 * hh + c] = __fmaf_rn(u0, sxr, acc[32 * hh + c]);
+              acc[32 * hh + c + 1] = __fmaf_rn(u1, sxr, acc[32 * hh + c + 1]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) acc[32 * hh + c] = __fadd_rn(acc[32 * hh + c], __uint_as_float(P[c]));
+          }
+        }
+      }
+      if (!ok) break;
+      if (row < p.M) {
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          const int n = n0 + 64 * ch + c;
+          if (n >= p.N) break;
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = __fadd_rn(acc[c + e], n + e < p.N ? __ldg(p.bias + n + e) : 0.0f);
+          if (n + 8 <= p.N && (p.N & 7) == 0) {
+            if constexpr (kF32Out) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + static_cast<size_t>(row) * p.N + n);
+              dst[0] = make_float4(y[0], y[1], y[2], y[3]);
+              dst[1] = make_float4(y[4], y[5], y[6], y[7]);
+            } else {
+              uint4 o;
+              __nv_bfloat162 h;
+              h = __floats2bfloat162_rn(y[0], y[1]); o.x = *reinterpret_cast<uint32_t*>(&h);
+              h = __floats2bfloat162_rn(y[2], y[3]); o.y = *reinterpret_cast<uint32_t*>(&h);
+              h = __floats2bfloat162_rn(y[4], y[5]); o.z = *reinterpret_cast<uint32_t*>(&h);
+              h = __floats2bfloat162_rn(y[6], y[7]); o.w = *reinterpret_cast<uint32_t*>(&h);
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + static_cast<size_t>(row) * p.N + n) = o;
+            }
+          } else {
+            for (int e = 0; e < 8 && n + e < p.N; ++e) {
+              if constexpr (kF32Out)
+                static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n + e] = y[e];
+              else
+                static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n + e] = __float2bfloat16_rn(y[e]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+teardown:
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < kI4Stages; ++s)
+      if (issued_mask & (1u << s)) mbar_wait_limited(&full[s], (issued_par >> s) & 1u, 200000000ull);
+  }
+  if (warp == 1) {
+    if (elect_one()) {
+      tc_commit(drain);  // the lane that issued the MMAs: arrives once they have finished
+      mbar_wait_limited(drain, 0, 200000000ull);
+    }
+    __syncwarp();
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.status, static_cast<int>(SVDQ_ERR_TIMEOUT));
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kI4TmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* lora_act, int M,
+                             void* Y, int out_dtype, cudaStream_t s) {
+  const int K = w->desc.K, N = w->desc.N;
+  const int m_pad = static_cast<int>(m_pad_of(M));
+  CUtensorMap tm_ap, tm_la;
+  // packed codes: M rows of K/2 bytes, 64-byte swizzled boxes of 128 rows x 64 bytes (128 K)
+  if (!encode_tmap_2d_swizzle(&tm_ap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K / 2, M, K / 2, 64, kTileM,
+                              CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (w->rank_pad > 0) {
+    if (!encode_tmap_2d(&tm_la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lora_act, w->rank_pad, M,
+                        static_cast<uint64_t>(w->rank_pad) * 4, 32, kTileM))
+      return cudaErrorInvalidValue;
+  } else {
+    tm_la = tm_ap;  // unused without a low-rank branch
+  }
+  I4Params p;
+  p.sx = static_cast<const __half*>(sx);
+  p.swp = w->swp;
+  p.bias = w->bias;
+  p.Y = Y;
+  p.status = w->status;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.m_pad = m_pad;
+  p.n_lora = w->rank_pad / 32;
+  p.n_pad = w->n_pad;
+  const int tiles = ((M + kTileM - 1) / kTileM) * ((N + kTileN - 1) / kTileN);
+  const int grid = std::min(tiles, num_sms(w->device));
+  auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_int4_kernel<true> : gemm_int4_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kI4Smem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kI4Threads, kI4Smem, s>>>(tm_ap, w->tm_qw8, tm_la, w->tm_l2, p);
+  return cudaGetLastError();
 }
 
 }  // namespace svdq

@@ -27,7 +27,15 @@ inline size_t int4_scale_bytes(int64_t rows_padded, int K) { return static_cast<
 struct WeightLayout {
   size_t qw, sw, l1s, l2, inv_lambda, bias, status, amax, total;
   size_t sw_bytes;
+  size_t qw8, swp;  // INT4 only (0 otherwise): unpacked int8 codes, float scale pairs
 };
+
+// INT4 working copies for the kind::i8 GEMM.  The tensor core takes 8-bit
+// operands, so the 4-bit codes are unpacked with one fixed permutation of K
+// inside every 8-value block: a packed word with nibbles k0..k7 becomes the
+// bytes k0 k2 k4 k6 k1 k3 k5 k7.  Both operands use it, so every dot
+// product (and every 64-group) is unchanged.
+constexpr float kI2FMagic = 12582912.0f;  // 1.5 * 2^23: bits(magic) + i = bits(magic + i), |i| < 2^22
 WeightLayout weight_layout(const svdq_layer_desc& d);
 
 }  // namespace svdq
@@ -48,11 +56,14 @@ struct svdq_weights {
   float* bias;
   int* status;    // written by the kernels when a bounded wait runs out
   uint32_t* amax; // scratch word of the preparation pass
+  int8_t* qw8;    // INT4: n_pad x K unpacked codes (K permuted as above); NVFP4: null
+  float2* swp;    // INT4: [K/64][n_pad] (s_w, -kI2FMagic * s_w); NVFP4: null
   int device;
   CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_sw;  // NVFP4 weight scales viewed as rows of 256 bytes, boxes of 8 rows (4 atoms)
   CUtensorMap tm_l1s; // bf16 L1s as 64-column chunks: boxes of all rank_pad rows x kQChunks chunks
+  CUtensorMap tm_qw8; // INT4: unpacked codes, 128-byte swizzled boxes of 128 rows x 128 K
 };
 
 namespace svdq {
@@ -75,6 +86,9 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
 // row of `row_bytes` stride, box {box_inner, box_rows}, 128-byte swizzle.
 bool encode_tmap_2d(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, bool swizzle128 = true);
+bool encode_tmap_2d_swizzle(CUtensorMap* tm, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                            uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                            CUtensorMapSwizzle swizzle);
 // A K-major bf16 matrix (rows x K, row pitch K * 2 bytes) seen as 64-column
 // chunks: dims {64, rows, K / 64}.  A {64, box_rows, box_chunks} box lands
 // in shared memory as box_chunks consecutive 128-byte-swizzled tiles of

@@ -140,6 +140,31 @@ __global__ void quantize_weights_kernel(const float* __restrict__ W, const float
   if (valid) *reinterpret_cast<uint2*>(qw + static_cast<size_t>(n) * (K / 2) + k0 / 2) = make_uint2(lo, hi);
 }
 
+// INT4 working copies: unpacked codes (K permuted within 8-value blocks,
+// rows N..n_pad zero) and the float scale pairs (s_w, -kI2FMagic s_w).
+__global__ void int4_unpack_kernel(const uint8_t* __restrict__ qw, const __half* __restrict__ sw, int N, int K,
+                                   int64_t n_pad, int8_t* __restrict__ qw8, float2* __restrict__ swp) {
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  const size_t blocks = static_cast<size_t>(n_pad) * (K / 8);
+  if (i < blocks) {
+    const int64_t n = static_cast<int64_t>(i / (K / 8));
+    const int j = static_cast<int>(i % (K / 8));
+    uint2 out = make_uint2(0u, 0u);
+    if (n < N) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + static_cast<size_t>(n) * (K / 2) + 4 * j);
+      // nibble -> signed byte without carries between bytes: ((v ^ 8) + 0x78) ^ 0x80
+      out.x = (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+      out.y = ((((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+    }
+    *reinterpret_cast<uint2*>(qw8 + static_cast<size_t>(n) * K + 8 * j) = out;
+  }
+  const size_t pairs = static_cast<size_t>(K / 64) * n_pad;
+  if (i < pairs) {
+    const float s = __half2float(sw[i]);
+    swp[i] = make_float2(s, -kI2FMagic * s);  // exact: an fp16 significand times 3 * 2^22
+  }
+}
+
 __global__ void l1s_kernel(const uint16_t* __restrict__ L1, const float* __restrict__ inv, int K, int r, int r_pad,
                            uint16_t* __restrict__ l1s) {
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -185,6 +210,9 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
   } else {
     quantize_weights_kernel<true><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
         W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw));
+    const size_t work = std::max(static_cast<size_t>(w->n_pad) * (K / 8), static_cast<size_t>(K / 64) * w->n_pad);
+    int4_unpack_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(
+        w->qw, static_cast<const __half*>(w->sw), N, K, w->n_pad, w->qw8, w->swp);
   }
   if (rp > 0) {
     const size_t n1 = static_cast<size_t>(rp) * K;

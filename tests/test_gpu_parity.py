@@ -244,6 +244,52 @@ def test_gemm_exact_on_integer_grid(svdq):
     assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
 
 
+@pytest.mark.parametrize("out_dtype", [1, 0], ids=["f32", "bf16"])
+@pytest.mark.parametrize("name,wl,over", CASES, ids=[c[0] for c in CASES])
+def test_forward_parity_int4(svdq, name, wl, over, out_dtype):
+    li = _layer(wl, over)
+    ol = T.oracle_layer(li, precision="int4")
+    w, y = _forward_case(svdq, li, ol, "int4", out_dtype)
+    ref = V.forward(li.x, ol.prep)
+    _assert_y(y, ref, out_dtype)
+
+
+def test_int4_gemm_exact_on_integer_grid(svdq):
+    """INT4 counterpart of the exactness pin: lambda = 1, rank 0, integer
+    codes and power-of-two fp16 scales make every partial sum an fp32-exact
+    value, so the kind::i8 product with its per-group scaling must equal the
+    oracle bit for bit.  This pins the nibble unpacking, the K permutation
+    inside 8-value blocks (the same on both operands) and both scale layouts.
+    K = 576 is an odd number of 64-groups (a half-filled last ring stage)."""
+    rng = np.random.default_rng(9)
+    M, K, N = 200, 576, 320
+    pow2 = np.array([0.25, 0.5, 1.0, 2.0])
+    # weights: every 64-group holds a 7 (amax = 7 s) so that the codes are W / s exactly
+    q_w = rng.integers(-7, 8, size=(N, K))
+    q_w[:, ::64] = 7
+    s_w = rng.choice(pow2, size=(N, K // 64))
+    W = (q_w * np.repeat(s_w, 64, axis=1)).astype(np.float32)
+    li = synth.LayerInputs(synth.WORKLOADS["tiny"], 0, np.zeros((M, K), np.uint16), np.zeros((M, K), np.float32), W,
+                           T.bf16_bits(np.zeros(N)), np.zeros(N, np.float32))
+    ol = T.oracle_layer(li, precision="int4", rank=0, lam=np.ones(K, np.float32))
+    assert np.array_equal(ol.prep.qw.astype(np.int64), q_w)
+    w = T.gpu_prepare(svdq, li, ol, "int4")
+    codes = rng.integers(-8, 8, size=(M, K)).astype(np.int8)
+    sx = rng.choice(pow2, size=(M, K // 64)).astype(np.float16)
+    mp = (M + 127) // 128 * 128
+    sx_dev = np.zeros((K // 64, mp), np.float16)
+    sx_dev[:, :M] = sx.T
+    qx = torch.from_numpy(F.pack_nibbles((codes.astype(np.int16) & 0xF).astype(np.uint8))).cuda()
+    sxt = torch.from_numpy(sx_dev.view(np.uint16).astype(np.int16)).cuda()
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    svdq.svdq_w4a4_gemm_lora_up(w, qx, sxt, 1.0, None, M, Y, 1)
+    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(w) == 0
+    act = V.ActQuant(codes, sx, np.zeros((M, 0)))
+    ref = V.forward_from_codes(act, ol.prep)
+    assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
+
+
 def test_argument_errors(svdq):
     li = _layer("tiny", {})
     ol = T.oracle_layer(li)
