@@ -15,8 +15,8 @@
 //               into int8 in the 128-byte-swizzled layout of the MMA operand
 //               (same K permutation as the prepared weights).
 //   warp 1      TMEM owner and MMA issuer: per group two kind::i8 MMAs
-//               (K = 32) into one of two int32 accumulators (128 columns
-//               each), so a group's MMAs overlap the previous group's
+//               (K = 32) into one of four int32 accumulators (128 columns
+//               each), so the MMAs run up to three groups ahead of the
 //               scaling; per tile four kind::tf32 MMAs of the lora-up into
 //               the next accumulator, as one more "group" of scale 1.
 //   warps 6-13  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM lane
@@ -46,10 +46,17 @@ constexpr int kA8Bytes = kTileM * 128;   // unpacked
 constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes
 constexpr int kI4StageBytes = kApBytes + kA8Bytes + kB8Bytes;  // 40 KB
 constexpr int kConvWarps = 4;
-constexpr int kI4EpiWarps = 8;
+constexpr int kI4EpiWarps = 8;  // 4 lane quarters x 2 column halves
 constexpr int kI4Threads = 32 * (2 + kConvWarps + kI4EpiWarps);
-constexpr uint32_t kI4TmemCols = 256;  // two accumulators of 128 columns
-constexpr size_t kI4Smem = kI4Stages * kI4StageBytes + 1024 /*align*/ + 512 /*barriers*/;
+constexpr int kAccBufs = 4;  // int32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
+constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
+// Group scales reach the epilogue through a ring of kScaleSlots groups in
+// shared memory, each thread fetching its value kScaleAhead groups early
+// (one global load's latency is much longer than a group's work).
+constexpr int kScaleSlots = 8, kScaleAhead = 4;
+constexpr int kScaleOff = kI4Stages * kI4StageBytes;  // per slot: 128 float2 s_w pairs + 128 float s_x
+constexpr int kI4BarOff = kScaleOff + kScaleSlots * (kTileN * 8 + kTileM * 4);
+constexpr size_t kI4Smem = kI4BarOff + 512 /*barriers*/ + 1024 /*align*/;
 static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 static_assert(kI4Smem <= 232448, "shared memory budget");
 
@@ -82,12 +89,14 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                      const I4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4Stages * kI4StageBytes);
+  float2* sc_sw = reinterpret_cast<float2*>(smem + kScaleOff);                          // [slots][128]
+  float* sc_sx = reinterpret_cast<float*>(smem + kScaleOff + kScaleSlots * kTileN * 8);  // [slots][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
   uint64_t* conv = full + kI4Stages;      // activation codes unpacked (4 converter warps)
   uint64_t* empty = conv + kI4Stages;     // MMAs done with the stage
-  uint64_t* acc_full = empty + kI4Stages;  // [2]
-  uint64_t* acc_empty = acc_full + 2;      // [2], 8 epilogue warps
-  uint64_t* drain = acc_empty + 2;
+  uint64_t* acc_full = empty + kI4Stages;      // [kAccBufs]
+  uint64_t* acc_empty = acc_full + kAccBufs;   // [kAccBufs], 8 epilogue warps
+  uint64_t* drain = acc_empty + kAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -105,7 +114,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       mbar_init(&conv[s], kConvWarps);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kI4EpiWarps);
     }
@@ -185,17 +194,21 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     // --------------------------------------------- MMA issuer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t gcount = 0;  // accumulator uses so far: buffer gcount & 1, its use gcount >> 1
+    // conv[s] completes once per K stage of slot s only (lora stages skip the
+    // converters), so its parity is tracked per slot, not with the ring phase
+    uint32_t conv_par = 0;
+    uint32_t gcount = 0;  // accumulator uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait_warp(&conv[stage], phase, abort_flag)) goto teardown;
+        if (!mbar_wait_warp(&conv[stage], (conv_par >> stage) & 1u, abort_flag)) goto teardown;
+        conv_par ^= 1u << stage;
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * kI4StageBytes + kApBytes);
         const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
         const int ng = min(2, groups - 2 * kb);
         for (int gi = 0; gi < ng; ++gi, ++gcount) {
-          const uint32_t buf = gcount & 1;
-          if (!mbar_wait_warp(&acc_empty[buf], ((gcount >> 1) & 1) ^ 1, abort_flag)) goto teardown;
+          const uint32_t buf = gcount % kAccBufs;
+          if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
           tc_fence_after();
           if (elect_one()) {
 #pragma unroll
@@ -210,8 +223,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
       }
       if (p.n_lora > 0) {  // the lora-up as one more accumulator use, of scale 1
-        const uint32_t buf = gcount & 1;
-        if (!mbar_wait_warp(&acc_empty[buf], ((gcount >> 1) & 1) ^ 1, abort_flag)) goto teardown;
+        const uint32_t buf = gcount % kAccBufs;
+        if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
         for (int j = 0; j < p.n_lora; ++j) {
           if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
           tc_fence_after();
@@ -233,45 +246,89 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    const int q4 = warp & 3;                     // TMEM lane quarter: rows 32 q4 .. + 31
-    const int ch = (warp - 2 - kConvWarps) >> 2;  // columns 64 ch .. + 63
+    // warp w owns rows 32 (w % 4) .. + 31 (its TMEM lane quarter) and 64
+    // columns.  A group's 128 s_w pairs and 128 s_x reach it through a ring
+    // of kScaleSlots entries in shared memory, one value per thread and entry,
+    // fetched kScaleAhead entries early.  The ring runs over the CTA's whole
+    // stream of (tile, group) pairs, index t, slot t % kScaleSlots: a thread
+    // writes entry t + kScaleAhead only after passing barrier t - 1, when every
+    // reader of entry t - kScaleAhead (same slot) is done.
+    const int q4 = warp & 3;
+    const int ch = (warp - 2 - kConvWarps) >> 2;         // columns 64 ch .. + 63
+    const int et = (warp - 2 - kConvWarps) * 32 + lane;  // 0 .. 255: s_w pair (< 128) or s_x
     const int r = 32 * q4 + lane;
     uint32_t gcount = 0;
     bool ok = true;
+    int f_tile = blockIdx.x, f_g = 0;  // the fetch cursor walks the stream in order
+    auto fetch = [&]() -> float2 {
+      float2 v = make_float2(0.0f, 0.0f);
+      if (f_tile < num_tiles) {
+        if (et < kTileN)
+          v = __ldg(p.swp + static_cast<size_t>(f_g) * p.n_pad + (f_tile / num_m) * kTileN + et);
+        else
+          v.x = __half2float(p.sx[static_cast<size_t>(f_g) * p.m_pad + (f_tile % num_m) * kTileM + et - kTileN]);
+        if (++f_g == groups) {
+          f_g = 0;
+          f_tile += gridDim.x;
+        }
+      }
+      return v;
+    };
+    auto put = [&](int slot, float2 v) {
+      if (et < kTileN)
+        sc_sw[slot * kTileN + et] = v;
+      else
+        sc_sx[slot * kTileM + et - kTileN] = v.x;
+    };
+    static_assert(kScaleAhead == 4 && kScaleSlots == 8, "queue depth");
+    for (int t = 0; t < kScaleAhead; ++t) put(t, fetch());
+    float2 q0 = fetch(), q1 = fetch(), q2 = fetch(), q3 = fetch();
+    uint32_t ti = 0;  // stream index of the next group (wraps harmlessly: slots are ti % 8)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
       const int row = m0 + r;
       float acc[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
-      for (int g = 0; g < groups + (p.n_lora > 0 ? 1 : 0); ++g, ++gcount) {
-        const uint32_t buf = gcount & 1;
-        if (!mbar_wait(&acc_full[buf], (gcount >> 1) & 1, abort_flag)) { ok = false; break; }
+      const int uses = groups + (p.n_lora > 0 ? 1 : 0);
+      for (int g = 0; g < uses; ++g, ++gcount) {
+        int sb = 0;
+        if (g < groups) {
+          put((ti + kScaleAhead) % kScaleSlots, q0);  // past the stream's end: harmless zeros
+          named_bar_sync(1, 32 * kI4EpiWarps);       // publishes entry ti
+          q0 = q1;
+          q1 = q2;
+          q2 = q3;
+          q3 = fetch();
+          sb = static_cast<int>(ti % kScaleSlots);
+          ++ti;
+        }
+        const uint32_t buf = gcount % kAccBufs;
+        if (!mbar_wait(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const bool lora = g == groups;
-        const float sxr = lora ? 1.0f : __half2float(p.sx[static_cast<size_t>(g) * p.m_pad + row]);
-        const float4* swq = reinterpret_cast<const float4*>(p.swp + static_cast<size_t>(lora ? 0 : g) * p.n_pad + n0 + 64 * ch);
+        const float sxr = sc_sx[sb * kTileM + r];
+        const float4* swq = reinterpret_cast<const float4*>(sc_sw + sb * kTileN + 64 * ch);  // broadcast
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time
           uint32_t P[32];
           tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + buf * kTileN + 64 * ch + 32 * hh, P);
           tmem_ld_wait();
-          if (hh == 1) {  // both halves are in registers: the accumulator is free
+          if (hh == 1) {  // both halves read: the accumulator is free
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
-          if (!lora) {
+          if (g < groups) {
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              const float4 t = __ldg(swq + (32 * hh + c) / 2);  // (s_w, -magic s_w) of two columns
+              const float4 t = swq[(32 * hh + c) / 2];  // (s_w, -magic s_w) of two columns
               // RN(P s_w) exactly: bits(magic) + P is the float magic + P
               const float u0 = __fmaf_rn(__int_as_float(static_cast<int>(P[c]) + 0x4B400000), t.x, t.y);
               const float u1 = __fmaf_rn(__int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000), t.z, t.w);
               acc[32 * hh + c] = __fmaf_rn(u0, sxr, acc[32 * hh + c]);
               acc[32 * hh + c + 1] = __fmaf_rn(u1, sxr, acc[32 * hh + c + 1]);
             }
-          } else {
+          } else {  // the lora-up, fp32
 #pragma unroll
             for (int c = 0; c < 32; ++c) acc[32 * hh + c] = __fadd_rn(acc[32 * hh + c], __uint_as_float(P[c]));
           }

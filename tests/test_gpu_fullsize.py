@@ -61,3 +61,42 @@ def test_full_size_nvfp4(svdq, workload):
             assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
         assert np.all(np.isfinite(Y.float().cpu().numpy()))
     assert svdq.svdq_device_status(w) == 0
+
+
+def test_full_size_int4(svdq):
+    """The INT4 configuration (four images: 18432 x 3072 -> 3072, rank 32)
+    at full size: every CTA of the persistent INT4 GEMM runs many tiles."""
+    li = synth.make_layer("int4", 4)
+    M, K, N = li.shape.M, li.shape.K, li.shape.N
+    ol = T.oracle_layer(li, precision="int4")
+    w = T.gpu_prepare(svdq, li, ol, "int4")
+    h = T.weights_to_host(w)
+    assert np.array_equal(T.unpack_codes(h["qw"]), (ol.prep.qw.astype(np.int16) & 0xF).astype(np.uint8))
+    sw = h["sw"].view(np.float16).reshape(K // 64, h["n_pad"])[:, :N].T
+    assert np.array_equal(sw.view(np.uint16), ol.prep.sw.view(np.uint16))
+
+    X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, 1.0)
+    rows = np.sort(np.random.default_rng(8).choice(M, SAMPLE_ROWS, replace=False))
+    act = V.quantize_activations(li.x[rows], ol.prep)
+    codes = T.nibbles_to_int(T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2)))
+    assert np.array_equal(codes[rows], act.qx)
+    mp = (M + 127) // 128 * 128
+    sxh = sx.cpu().numpy().view(np.float16).reshape(K // 64, mp)
+    assert np.array_equal(sxh[:, rows].T.view(np.uint16), act.sx.view(np.uint16))
+
+    ref = V.forward_from_codes(act, ol.prep)
+    rms = np.sqrt(np.mean(ref ** 2))
+    for out_dtype in (1, 0):
+        Y = torch.empty((M, N), dtype=torch.float32 if out_dtype else torch.bfloat16, device="cuda")
+        svdq.svdq_w4a4_gemm_lora_up(w, qx, sx, 1.0, la, M, Y, out_dtype)
+        torch.cuda.synchronize()
+        y = Y.float().cpu().numpy()[rows].astype(np.float64)
+        d = y - ref
+        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F
+        if out_dtype:
+            assert np.abs(d).max() <= MAX_ABS * rms
+        else:
+            half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
+            assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
+        assert np.all(np.isfinite(Y.float().cpu().numpy()))
+    assert svdq.svdq_device_status(w) == 0

@@ -44,6 +44,8 @@ CASES = [
     ("partial_k_n_rank64", "mlp_up", dict(M=129, K=320, N=144, rank=64)),
     ("rank0", "stack_out", dict(M=200, K=512, N=512, rank=0)),
     ("rank8", "mlp_down", dict(M=77, K=768, N=272, rank=8)),
+    # more output tiles than CTAs: the persistent GEMMs wrap around the tile list
+    ("many_tiles", "qkv", dict(M=2048, K=320, N=2560)),
 ]
 
 
