@@ -293,6 +293,94 @@ def run_ours(args, li, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_stack(args, rank, world, local_rank):
+    """One denoising step of a random-init stack of `--blocks` MMDiT-style
+    blocks (QKV 3072->9216, out 3072->3072, MLP up 3072->12288, down
+    12288->3072; M = 4608 tokens, rank 32, NVFP4): every linear through
+    svdq_linear_forward, each with its own seeded weights, input and
+    calibration (inputs are not chained: attention and norms are not part of
+    the layer).  Weights and inputs are drawn on the GPU; preparation is
+    untimed.  One L2 read-flush before each timed step."""
+    import torch
+    import synth
+    from bit_diffusion_transformer_svdq_b200 import svdq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    svdq.load_library()
+    stream = torch.cuda.current_stream()
+    M = synth.WORKLOADS["stack_qkv"].M
+    layers = []
+    for blk in range(args.blocks):
+        for j, name in enumerate(synth.STACK_LAYERS):
+            shp = synth.WORKLOADS[name]
+            K, N, r = shp.K, shp.N, shp.rank
+            g = torch.Generator(device=dev)
+            g.manual_seed(synth.stack_seed(blk, j))
+            W = torch.randn(N, K, generator=g, device=dev) * 0.02
+            Xf = torch.randn(M, K, generator=g, device=dev)
+            Xf[:, torch.randperm(K, generator=g, device=dev)[:4]] *= 50.0  # the outlier channels
+            X = Xf.to(torch.bfloat16).view(torch.int16)
+            b = (torch.randn(N, generator=g, device=dev) * 0.01).to(torch.bfloat16).view(torch.int16)
+            lam = torch.empty(K, dtype=torch.float32, device=dev)
+            scratch = torch.empty(2 * K, dtype=torch.float32, device=dev)
+            svdq.svdq_smoothing_lambda(X, W, lam, scratch)
+            U, S, Vv = torch.svd_lowrank((W * lam[None, :]).t(), q=r + 16, niter=4)
+            L1 = (U[:, :r] * S[None, :r]).t().contiguous().to(torch.bfloat16).view(torch.int16)
+            L2 = Vv[:, :r].contiguous().to(torch.bfloat16).view(torch.int16)
+            w = svdq.prepare_layer(W, lam, L1, L2, b, r)
+            gx_t = torch.empty(1, dtype=torch.float32, device=dev)
+            svdq.svdq_act_global_scale(w, X, gx_t)
+            layers.append((w, X, float(gx_t.item()), N, K))
+            del W, Xf, U, S, Vv
+    torch.cuda.empty_cache()
+    ws_bytes = max(svdq.svdq_workspace_bytes(w, M) for (w, _, _, _, _) in layers[:4])
+    ws = svdq.alloc_workspace(layers[0][0], M, dev, nbytes=ws_bytes)
+    Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (_, _, _, N, _) in layers[:4]}
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def step():
+        for (w, X, gx, N, _) in layers:
+            svdq.svdq_linear_forward(w, X, M, gx, Ys[N], ws, ws.numel(), svdq.SVDQ_OUT_BF16, stream)
+
+    for _ in range(args.warmup):
+        flush.sum()
+        step()
+    torch.cuda.synchronize()
+    assert all(svdq.svdq_device_status(w) == 0 for (w, _, _, _, _) in layers)
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    time.sleep(0.1)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ts = []
+    for _ in range(args.steps):
+        flush.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    _barrier(world)
+    clocks = sampler.stop(t_wall0, time.time())
+    assert all(svdq.svdq_device_status(w) == 0 for (w, _, _, _, _) in layers)
+    t_ms = _allreduce_max(sum(a.elapsed_time(b) for a, b in ts) / len(ts), world, dev)
+    flops = sum(2.0 * M * N * K for (_, _, _, N, K) in layers)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "fused SVDQuant W4A4 linear effective TOPS, one denoising step of the block stack",
+            "value": world * flops / (t_ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+            "config": {"workload": f"{args.blocks} blocks x 4 linears (QKV, out, MLP up, down), M={M}, rank 32, nvfp4",
+                       "linears": len(layers), "l2": "flushed (256 MiB read) once before each step",
+                       "parallelism": f"replicas x{world}"},
+            "gpu_launches": 2 * len(layers) * args.steps, "clocks": clocks}), flush=True)
+
+
 def _barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -317,6 +405,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=None, help="override M (smaller profiling cases only)")
+    ap.add_argument("--workload", default="qkv", choices=["qkv", "stack"],
+                    help="qkv: the single-layer bench line; stack: one denoising step of the block stack")
+    ap.add_argument("--blocks", type=int, default=57, help="blocks of the stack workload")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -335,6 +426,14 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.workload == "stack":
+        try:
+            run_stack(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+        return
     li = synth.make_layer(WORKLOAD, SEED, **({"M": args.rows} if args.rows else {}))
     try:
         run_ours(args, li, rank, world, local_rank)

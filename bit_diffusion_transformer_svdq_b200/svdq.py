@@ -234,8 +234,10 @@ def prepare_layer(W: torch.Tensor, lam: torch.Tensor, L1: torch.Tensor | None, L
     return svdq_prepare_weights(desc, W, lam, L1, L2, bias, storage, stream)
 
 
-def alloc_workspace(w: Weights, M: int, device) -> torch.Tensor:
-    n = svdq_workspace_bytes(w, M)
+def alloc_workspace(w: Weights, M: int, device, nbytes: int | None = None) -> torch.Tensor:
+    """A 1024-aligned device workspace of svdq_workspace_bytes(w, M) bytes
+    (or `nbytes`, e.g. the largest over several layers sharing it)."""
+    n = svdq_workspace_bytes(w, M) if nbytes is None else nbytes
     buf = torch.empty(n + 1024, dtype=torch.uint8, device=device)
     off = (-buf.data_ptr()) % 1024
     return buf[off:off + n]

@@ -100,3 +100,34 @@ def test_full_size_int4(svdq):
             assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
         assert np.all(np.isfinite(Y.float().cpu().numpy()))
     assert svdq.svdq_device_status(w) == 0
+
+
+def test_stack_block_through_forward(svdq):
+    """One block of the 57-block denoising stack at full size (QKV 3072 ->
+    9216, out 3072 -> 3072, MLP up 3072 -> 12288, down 12288 -> 3072; M =
+    4608, rank 32, NVFP4), every linear through svdq_linear_forward with the
+    per-layer seeds of the stack: sampled codes and scales bit-exact, sampled
+    Y rows within the bf16-output tolerance."""
+    for layer, name in enumerate(synth.STACK_LAYERS):
+        li = synth.make_layer(name, synth.stack_seed(0, layer))
+        M, K, N = li.shape.M, li.shape.K, li.shape.N
+        ol = T.oracle_layer(li)
+        w = T.gpu_prepare(svdq, li, ol)
+        rows = np.sort(np.random.default_rng(100 + layer).choice(M, 64, replace=False))
+        act = V.quantize_activations(li.x[rows], ol.prep, ol.gx)
+        X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
+        codes = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
+        assert np.array_equal(codes[rows], act.qx), name
+        assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K)[rows], act.sx), name
+        ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        svdq.svdq_linear_forward(w, X, M, float(ol.gx), Y, ws, ws.numel(), 0)
+        torch.cuda.synchronize()
+        assert svdq.svdq_device_status(w) == 0
+        ref = V.forward_from_codes(act, ol.prep, ol.gx)
+        y = Y.float().cpu().numpy()[rows].astype(np.float64)
+        d = y - ref
+        rms = np.sqrt(np.mean(ref ** 2))
+        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F, name
+        half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
+        assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp), name
