@@ -73,6 +73,7 @@ _SIGS = {
     "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _P, _I, _F, _P, _I, _P]),
     "svdq_device_status": (_I, [_P, _P]),
+    "svdq_selftest_bounded_wait": (_I, [_P]),
 }
 
 
@@ -214,6 +215,12 @@ def svdq_linear_forward_noalloc(w: Weights, X, M: int, g_x: float, Y, out_dtype:
 
 def svdq_device_status(w: Weights, stream=None) -> int:
     return load_library().svdq_device_status(w.handle, _stream(stream))
+
+
+def svdq_selftest_bounded_wait(stream=None) -> int:
+    """Runs the bounded-wait self-test kernel; a healthy library returns
+    SVDQ_ERR_TIMEOUT (6) after about two seconds."""
+    return load_library().svdq_selftest_bounded_wait(_stream(stream))
 
 
 # ----------------------------------------------------------------- helpers

@@ -229,6 +229,16 @@ SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const ui
  * SVDQ_ERR_TIMEOUT, else SVDQ_OK (or SVDQ_ERR_CUDA if the sync failed). */
 SVDQ_API svdq_status svdq_device_status(const svdq_weights* w, void* stream);
 
+/* Self-test of the failure path every kernel shares (no counterpart in the
+ * pages).  Launches a one-thread kernel whose bounded wait on an mbarrier
+ * that nothing arrives on runs out at its limit (2 s of globaltimer) and
+ * records SVDQ_ERR_TIMEOUT; synchronises `stream` and returns that status.
+ * The kernel neither faults nor traps, so the context stays usable: a
+ * healthy library returns SVDQ_ERR_TIMEOUT here (SVDQ_OK would mean the
+ * wait completed without its arrival, SVDQ_ERR_CUDA a launch or copy
+ * failure, SVDQ_ERR_UNSUPPORTED_DEVICE a device that is not sm_100). */
+SVDQ_API svdq_status svdq_selftest_bounded_wait(void* stream);
+
 #ifdef __cplusplus
 }
 #endif
