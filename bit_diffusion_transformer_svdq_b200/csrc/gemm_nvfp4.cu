@@ -15,8 +15,10 @@
 //               tf32 lora-up MMAs into the accumulator, then per K step the
 //               scale copies to TMEM (tcgen05.cp) and the block-scaled
 //               kind::mxf4nvf4 MMAs (K = 64 each).
-//   warps 2-9   epilogue (both CTAs): drain the CTA's 128 x 256 fp32 rows
-//               from TMEM, release them to the MMA issuer, then
+//   warps 2-17  epilogue (both CTAs): drain the CTA's 128 x 256 fp32 rows
+//               from TMEM (16 warps, 64 columns each, so the drain that
+//               holds up the next tile is short), release them to the MMA
+//               issuer with one arrival per CTA, then
 //               y = acc * RN32(g_x g_w) + b (the tile's bias read once into
 //               shared memory), written as bf16 or fp32 into 128-byte-
 //               swizzled staging boxes and stored by TMA in whole lines.
@@ -47,11 +49,12 @@ constexpr int kBBytes = 128 * BK / 2;                                  // 16 KB 
 constexpr int kSfaBytes = 128 * BK / 16;                               // 2 KB
 constexpr int kSfbBytes = 256 * BK / 16;                               // 4 KB (all 256 N)
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;  // 38 KB
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;                       // 4 TMEM lane quarters x 4 column quarters
+constexpr int kColsPerWarp = BN * 4 / kEpiWarps;    // 64
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0, kColSf = 256, kSfSlotCols = 48;
-constexpr int kStagingPerWarp = 8192;  // two 32-row x 128-byte output boxes per epilogue warp
+constexpr int kStagingPerWarp = 4096;  // one 32-row x 128-byte output box per epilogue warp
 constexpr int kStagingOff = kStages * kStageBytes;
 constexpr int kBiasOff = kStagingOff + kEpiWarps * kStagingPerWarp;  // 2 x 256 floats
 constexpr int kBarOff = kBiasOff + 2 * BN * 4;
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * kEpiWarps);
+    mbar_init(acc_empty, 2);  // one arrival per CTA, after all its epilogue warps have drained
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -228,54 +231,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // Warp (quarter, half) owns rows quarter*32 .. +31 (its TMEM lane
-    // quarter) and columns half*128 .. +127 of the CTA's 128 x 256 tile.
+    // Warp (quarter, part) owns rows quarter*32 .. +31 (its TMEM lane
+    // quarter) and columns part*64 .. +63 of the CTA's 128 x 256 tile.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    const int et = (warp - 2) * 32 + lane;  // 0..255 over the epilogue warps
+    const int part = (warp - 2) >> 2;
+    const int et = (warp - 2) * 32 + lane;  // 0..511 over the epilogue warps
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    uint8_t* const stg = smem + kStagingOff + (warp - 2) * kStagingPerWarp;  // 128-byte-swizzled boxes
+    uint8_t* const stg = smem + kStagingOff + (warp - 2) * kStagingPerWarp;  // a 128-byte-swizzled box
     uint32_t acc_phase = 0;
     int tcount = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
       const int m0 = (tile % num_m) * BM + 128 * static_cast<int>(rank), n0 = (tile / num_m) * BN;
       // the tile's 256 bias values, once, into this tile's half of the double buffer
       float* bias_t = bias_s + (tcount & 1) * BN;
-      bias_t[et] = n0 + et < p.N ? __ldg(p.bias + n0 + et) : 0.0f;
+      if (et < BN) bias_t[et] = n0 + et < p.N ? __ldg(p.bias + n0 + et) : 0.0f;
       named_bar_sync(1, 32 * kEpiWarps);
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
       acc_phase ^= 1;
       tc_fence_after();
-      uint32_t v[128];  // this warp's 32 rows x 128 columns, one load
-      tmem_ld128(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColAcc + half * 128, v);
+      uint32_t v[kColsPerWarp];  // this warp's 32 rows x 64 columns, one load
+      tmem_ld64(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kColAcc + part * kColsPerWarp, v);
       tmem_ld_wait();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc_empty_leader);  // the accumulator is free for the next tile
+      // once every epilogue warp of this CTA holds its columns, one arrival
+      // (local or remote) frees the accumulator for the next tile
+      named_bar_sync(2, 32 * kEpiWarps);
+      if (warp == 2 && lane == 0) mbar_arrive_cluster(acc_empty_leader);
 
       const int row = m0 + quarter * 32 + lane;
-      const float* bb = bias_t + half * 128;
+      const float* bb = bias_t + part * kColsPerWarp;
       if (p.tma_store) {
-        // y rows into 128-byte-wide swizzled boxes (32 rows each), then TMA
-        // stores of whole lines; rows past M / columns past N are clipped
+        // y rows into a 128-byte-wide swizzled box (32 rows), then a TMA
+        // store of whole lines per box; rows past M / columns past N are clipped
         constexpr int kColsPerBox = kF32Out ? 32 : 64;
-        constexpr int kPasses = kF32Out ? 2 : 1;  // 64 or 128 columns per staging fill
+        constexpr int kPasses = kColsPerWarp / kColsPerBox;
 #pragma unroll
         for (int pass = 0; pass < kPasses; ++pass) {
-          if (lane == 0) bulk_wait_read_all();  // the previous stores no longer read the boxes
+          if (lane == 0) bulk_wait_read_all();  // the previous store no longer reads the box
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 128 / kPasses; j += 4) {
-            const int col = pass * (128 / kPasses) + j;  // within the warp's 128 columns
+          for (int j = 0; j < kColsPerBox; j += 4) {
+            const int col = pass * kColsPerBox + j;  // within the warp's columns
             const uint32_t* a = &v[col];
             const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(a[0]), p.gxgw), bb[col]);
             const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(a[1]), p.gxgw), bb[col + 1]);
             const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(a[2]), p.gxgw), bb[col + 2]);
             const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(a[3]), p.gxgw), bb[col + 3]);
-            const int lc = col - pass * (128 / kPasses);   // column within this fill
-            const int box = lc / kColsPerBox;
-            const int byte = (lc % kColsPerBox) * (kF32Out ? 4 : 2);  // within the box's 128-byte row
-            uint8_t* line = stg + box * 4096 + lane * 128;
+            const int byte = j * (kF32Out ? 4 : 2);  // within the box's 128-byte row
+            uint8_t* line = stg + lane * 128;
             if constexpr (kF32Out) {
               *reinterpret_cast<float4*>(line + (((byte >> 4) ^ (lane & 7)) << 4)) = make_float4(y0, y1, y2, y3);
             } else {
@@ -287,35 +290,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-#pragma unroll
-            for (int b = 0; b < 128 / kPasses / kColsPerBox; ++b)
-              tma_store_2d(&tm_y, stg + b * 4096, n0 + half * 128 + pass * (128 / kPasses) + b * kColsPerBox,
-                           m0 + quarter * 32);
+            tma_store_2d(&tm_y, stg, n0 + part * kColsPerWarp + pass * kColsPerBox, m0 + quarter * 32);
             bulk_commit_group();
           }
         }
       } else if (row < p.M) {
         // rows whose byte length is not a multiple of 16: plain stores
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int col = 32 * c + i;
-            const int n = n0 + half * 128 + col;
-            if (n < p.N) {
-              const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
-              if constexpr (kF32Out)
-                static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
-              else
-                static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n] = __float2bfloat16_rn(y);
-            }
+        for (int col = 0; col < kColsPerWarp; ++col) {
+          const int n = n0 + part * kColsPerWarp + col;
+          if (n < p.N) {
+            const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
+            if constexpr (kF32Out)
+              static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
+            else
+              static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n] = __float2bfloat16_rn(y);
           }
         }
       }
     }
     if (lane == 0) bulk_wait_all();  // every store of this warp has landed
   }
-
 
 teardown:
   __syncthreads();
