@@ -20,8 +20,8 @@
 //               holds up the next tile is short), release them to the MMA
 //               issuer with one arrival per CTA, then
 //               y = acc * RN32(g_x g_w) + b (the tile's bias read once into
-//               shared memory), written as bf16 or fp32 into 128-byte-
-//               swizzled staging boxes and stored by TMA in whole lines.
+//               shared memory), written as bf16 or fp32 into 64-byte-
+//               swizzled staging boxes and stored by TMA.
 // The lora-up shares the accumulator with the 4-bit product because
 // lora_act arrives pre-divided by g_x g_w.
 //
@@ -43,7 +43,7 @@ namespace {
 constexpr int BM = 256;  // rows of a pair tile (128 per CTA)
 constexpr int BN = 256;
 constexpr int BK = 256;  // fp4 elements per ring stage (128 bytes per row)
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kABytes = 128 * BK / 2;                                  // 16 KB
 constexpr int kBBytes = 128 * BK / 2;                                  // 16 KB (this CTA's N half)
 constexpr int kSfaBytes = 128 * BK / 16;                               // 2 KB
@@ -54,7 +54,10 @@ constexpr int kColsPerWarp = BN * 4 / kEpiWarps;    // 64
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = 0, kColSf = 256, kSfSlotCols = 48;
-constexpr int kStagingPerWarp = 4096;  // one 32-row x 128-byte output box per epilogue warp
+// one 32-row x 64-byte output box per epilogue warp (64-byte swizzle): the
+// ring keeps five stages (190 KB of TMA loads in flight, which the L2 needs
+// to deliver a K step per MMA time)
+constexpr int kStagingPerWarp = 2048;
 constexpr int kStagingOff = kStages * kStageBytes;
 constexpr int kBiasOff = kStagingOff + kEpiWarps * kStagingPerWarp;  // 2 x 256 floats
 constexpr int kBarOff = kBiasOff + 2 * BN * 4;
@@ -261,9 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row = m0 + quarter * 32 + lane;
       const float* bb = bias_t + part * kColsPerWarp;
       if (p.tma_store) {
-        // y rows into a 128-byte-wide swizzled box (32 rows), then a TMA
-        // store of whole lines per box; rows past M / columns past N are clipped
-        constexpr int kColsPerBox = kF32Out ? 32 : 64;
+        // y rows into a 64-byte-wide swizzled box (32 rows; row r's 16-byte
+        // unit u at r * 64 + ((u ^ ((r >> 1) & 3)) << 4)), then a TMA store
+        // per box; rows past M / columns past N are clipped
+        constexpr int kColsPerBox = kF32Out ? 16 : 32;
         constexpr int kPasses = kColsPerWarp / kColsPerBox;
 #pragma unroll
         for (int pass = 0; pass < kPasses; ++pass) {
@@ -277,13 +281,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(a[1]), p.gxgw), bb[col + 1]);
             const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(a[2]), p.gxgw), bb[col + 2]);
             const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(a[3]), p.gxgw), bb[col + 3]);
-            const int byte = j * (kF32Out ? 4 : 2);  // within the box's 128-byte row
-            uint8_t* line = stg + lane * 128;
+            const int byte = j * (kF32Out ? 4 : 2);  // within the box's 64-byte row
+            uint8_t* line = stg + lane * 64;
+            const int unit = (byte >> 4) ^ ((lane >> 1) & 3);
             if constexpr (kF32Out) {
-              *reinterpret_cast<float4*>(line + (((byte >> 4) ^ (lane & 7)) << 4)) = make_float4(y0, y1, y2, y3);
+              *reinterpret_cast<float4*>(line + (unit << 4)) = make_float4(y0, y1, y2, y3);
             } else {
               __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1), h1 = __floats2bfloat162_rn(y2, y3);
-              *reinterpret_cast<uint2*>(line + (((byte >> 4) ^ (lane & 7)) << 4) + (byte & 15)) =
+              *reinterpret_cast<uint2*>(line + (unit << 4) + (byte & 15)) =
                   make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
             }
           }
@@ -368,8 +373,8 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   const uint64_t row_bytes = static_cast<uint64_t>(N) * (f32 ? 4 : 2);
   CUtensorMap tm_y = tm_a;
   p.tma_store = row_bytes % 16 == 0 &&
-                encode_tmap_2d(&tm_y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M,
-                               row_bytes, f32 ? 32 : 64, 32);
+                encode_tmap_2d_swizzle(&tm_y, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y,
+                                       N, M, row_bytes, f32 ? 16 : 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int pairs = std::min(tiles, num_sms(w->device) / 2);
   auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
