@@ -259,7 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // once every epilogue warp of this CTA holds its columns, one arrival
       // (local or remote) frees the accumulator for the next tile
       named_bar_sync(2, 32 * kEpiWarps);
-      if (warp == 2 && lane == 0) mbar_arrive_cluster(acc_empty_leader);
+      if (warp == 2 && lane == 0) {
+        // the loads above have completed (wait::ld), so the signal orders no
+        // memory access: the first CTA arrives locally, its peer remotely
+        // without a cluster-scope release (which cost ~1000 cycles per tile)
+        if (rank == 0) mbar_arrive(acc_empty);
+        else mbar_arrive_cluster_relaxed(acc_empty_leader);
+      }
 
       const int row = m0 + quarter * 32 + lane;
       const float* bb = bias_t + part * kColsPerWarp;
