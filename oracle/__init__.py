@@ -29,5 +29,7 @@ Modules:
   svd      - truncated SVD (LAPACK for small, subspace iteration for large)
   svdq     - smoothing factor, weight preparation, activation quantisation
              with lora-down, and the fp64 forward
+  qkv      - the attention prologue of the fused QKV projection (per-head
+             RMS normalisation of Q and K, rotary embedding)
 """
-from . import formats, quant, svd, svdq  # noqa: F401
+from . import formats, qkv, quant, svd, svdq  # noqa: F401
