@@ -306,8 +306,10 @@ svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X
   return from_cuda(launch_quantize(w, X, M, g_x, qx, sx, lora_act, static_cast<cudaStream_t>(stream)));
 }
 
-svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
-                                   const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream) {
+namespace {
+// Shared by the GEMM entry points: argument checks, then the launch.
+svdq_status gemm_entry(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x, const float* lora_act,
+                       int32_t M, const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* stream) {
   if (!w) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
@@ -321,8 +323,34 @@ svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, con
   if (st != SVDQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (w->desc.precision == SVDQ_NVFP4)
-    return from_cuda(launch_gemm_nvfp4(w, qx, static_cast<const uint8_t*>(sx), g_x, lora_act, M, Y, out_dtype, s));
-  return from_cuda(launch_gemm_int4(w, qx, sx, lora_act, M, Y, out_dtype, s));
+    return from_cuda(launch_gemm_nvfp4(w, qx, static_cast<const uint8_t*>(sx), g_x, lora_act, M, Y, out_dtype, pro, s));
+  return from_cuda(launch_gemm_int4(w, qx, sx, lora_act, M, Y, out_dtype, pro, s));
+}
+
+// The QKV prologue's limits (see svdq.h).
+svdq_status check_qkv(const svdq_weights* w, const svdq_qkv_prologue* pro) {
+  if (!w || !pro) return SVDQ_ERR_INVALID_ARG;
+  if (!pro->norm_q || !pro->norm_k || !pro->rope_cos || !pro->rope_sin) return SVDQ_ERR_INVALID_ARG;
+  if (!(pro->eps > 0.0f && pro->eps < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
+  if (pro->head_dim != 128 || pro->heads < 2 || (pro->heads & 1)) return SVDQ_ERR_SHAPE;
+  if (static_cast<int64_t>(w->desc.N) != 3LL * pro->heads * pro->head_dim) return SVDQ_ERR_SHAPE;
+  if (!aligned16(pro->norm_q) || !aligned16(pro->norm_k) || !aligned16(pro->rope_cos) || !aligned16(pro->rope_sin))
+    return SVDQ_ERR_ALIGNMENT;
+  return SVDQ_OK;
+}
+}  // namespace
+
+svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
+                                   const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream) {
+  return gemm_entry(w, qx, sx, g_x, lora_act, M, nullptr, Y, out_dtype, stream);
+}
+
+svdq_status svdq_w4a4_gemm_lora_up_qkv(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
+                                       const float* lora_act, int32_t M, const svdq_qkv_prologue* pro, void* Y,
+                                       int32_t out_dtype, void* stream) {
+  const svdq_status st = check_qkv(w, pro);
+  if (st != SVDQ_OK) return st;
+  return gemm_entry(w, qx, sx, g_x, lora_act, M, pro, Y, out_dtype, stream);
 }
 
 size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M) {
@@ -333,8 +361,10 @@ size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M) {
   return qx + sx + la;
 }
 
-svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
-                                int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+namespace {
+svdq_status forward_entry(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
+                          const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace, size_t ws_bytes,
+                          void* stream) {
   if (!w) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
@@ -347,7 +377,21 @@ svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_
   float* la = reinterpret_cast<float*>(sx + round_up(static_cast<int64_t>(svdq_act_scale_bytes(w, M)), 1024));
   svdq_status st = svdq_quantize_act_lora_down(w, X, M, g_x, qx, sx, w->rank_pad ? la : nullptr, stream);
   if (st != SVDQ_OK) return st;
-  return svdq_w4a4_gemm_lora_up(w, qx, sx, g_x, w->rank_pad ? la : nullptr, M, Y, out_dtype, stream);
+  return gemm_entry(w, qx, sx, g_x, w->rank_pad ? la : nullptr, M, pro, Y, out_dtype, stream);
+}
+}  // namespace
+
+svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
+                                int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  return forward_entry(w, X, M, g_x, nullptr, Y, out_dtype, workspace, ws_bytes, stream);
+}
+
+svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
+                                    const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace,
+                                    size_t ws_bytes, void* stream) {
+  const svdq_status st = check_qkv(w, pro);
+  if (st != SVDQ_OK) return st;
+  return forward_entry(w, X, M, g_x, pro, Y, out_dtype, workspace, ws_bytes, stream);
 }
 
 svdq_status svdq_device_status(const svdq_weights* w, void* stream) {

@@ -24,7 +24,11 @@
 //               product and adds RN(P s_w) s_x to its fp32 accumulator.
 //               RN(P s_w) is one FMA on the bit pattern magic + P (exact for
 //               |P| < 2^22; a group's |P| is at most 64 * 8 * 8), no
-//               int-to-float conversion.  Finally y = acc + b is stored.
+//               int-to-float conversion.  Finally y = acc + b is stored;
+//               the QKV variant first applies the attention prologue (per
+//               128-column head of Q and K: RMS normalisation, weight,
+//               rotary embedding), the two column halves of a row adding
+//               their sums of squares through shared memory.
 // The group rescale is CUDA-core work on every output element (three
 // operations per element per 64 K, against 64 MACs on the tensor core), so
 // this kernel is bound by it, not by the MMAs.
@@ -56,7 +60,8 @@ constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
 constexpr int kScaleSlots = 8, kScaleAhead = 4;
 constexpr int kScaleOff = kI4Stages * kI4StageBytes;  // per slot: 128 float2 s_w pairs + 128 float s_x
 constexpr int kI4BarOff = kScaleOff + kScaleSlots * (kTileN * 8 + kTileM * 4);
-constexpr size_t kI4Smem = kI4BarOff + 512 /*barriers*/ + 1024 /*align*/;
+constexpr int kI4RedOff = kI4BarOff + 512;  // QKV: one float per row of a head (4 x 32)
+constexpr size_t kI4Smem = kI4RedOff + 4 * 32 * 4 + 1024 /*align*/;
 static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 static_assert(kI4Smem <= 232448, "shared memory budget");
 
@@ -80,9 +85,17 @@ struct I4Params {
   int* status;
   int M, N, K, m_pad, n_lora;
   int64_t n_pad;
+  // QKV attention prologue (the kQkv variant only); a 128-column tile is
+  // one head of Q, K or V
+  const float* norm_q;
+  const float* norm_k;
+  const float* rope_cos;  // 64 x M, frequency-major
+  const float* rope_sin;
+  float eps;
+  int qk_cols;  // 2 * heads * 128; K starts at qk_cols / 2
 };
 
-template <bool kF32Out>
+template <bool kF32Out, bool kQkv>
 __global__ void __launch_bounds__(kI4Threads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_b8,
                      const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
@@ -91,6 +104,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float2* sc_sw = reinterpret_cast<float2*>(smem + kScaleOff);                          // [slots][128]
   float* sc_sx = reinterpret_cast<float*>(smem + kScaleOff + kScaleSlots * kTileN * 8);  // [slots][128]
+  float* red_s = reinterpret_cast<float*>(smem + kI4RedOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
   uint64_t* conv = full + kI4Stages;      // activation codes unpacked (4 converter warps)
   uint64_t* empty = conv + kI4Stages;     // MMAs done with the stage
@@ -335,6 +349,55 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         }
       }
       if (!ok) break;
+      if constexpr (kQkv) {
+        // y = acc + b in place (N is a multiple of 128 here), then in Q / K
+        // tiles the head's RMS normalisation and rotary embedding; the two
+        // column halves of a row add their sums of squares through shared
+        // memory (the lower half first).  Every epilogue warp works on the
+        // same tile, so the barriers are uniform; the slot is next written
+        // after the next tile's first scale barrier.
+        const int nc = n0 + 64 * ch;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) acc[c] = __fadd_rn(acc[c], __ldg(p.bias + nc + c));
+        if (n0 < p.qk_cols) {
+          float ss = 0.0f;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) ss = __fmaf_rn(acc[c], acc[c], ss);
+          float* slot = red_s + q4 * 32 + lane;
+          if (ch) *slot = ss;
+          named_bar_sync(2, 32 * kI4EpiWarps);
+          if (!ch) *slot = __fadd_rn(ss, *slot);
+          named_bar_sync(2, 32 * kI4EpiWarps);
+          const float rs = rsqrtf(__fmaf_rn(*slot, 1.0f / 128.0f, p.eps));
+          const float4* wn = reinterpret_cast<const float4*>((n0 < p.qk_cols / 2 ? p.norm_q : p.norm_k) + 64 * ch);
+          // frequency-major rotary tables: one line per frequency per warp
+          const bool in_rows = row < p.M;
+          const size_t trow = static_cast<size_t>(32 * ch) * p.M + (in_rows ? row : 0);
+          const float* ct = p.rope_cos + trow;
+          const float* st = p.rope_sin + trow;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {  // four pairs per step
+            float cc[4], sc[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              cc[j] = in_rows ? __ldg(ct + static_cast<size_t>(4 * q + j) * p.M) : 1.0f;
+              sc[j] = in_rows ? __ldg(st + static_cast<size_t>(4 * q + j) * p.M) : 0.0f;
+            }
+            const float4 w0 = __ldg(wn + 2 * q), w1 = __ldg(wn + 2 * q + 1);
+            // the head's scale folded into the weights: (y r) w = y (r w)
+            const float rw[8] = {__fmul_rn(rs, w0.x), __fmul_rn(rs, w0.y), __fmul_rn(rs, w0.z), __fmul_rn(rs, w0.w),
+                                 __fmul_rn(rs, w1.x), __fmul_rn(rs, w1.y), __fmul_rn(rs, w1.z), __fmul_rn(rs, w1.w)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = 8 * q + 2 * j;
+              const float a = __fmul_rn(acc[c], rw[2 * j]);
+              const float b = __fmul_rn(acc[c + 1], rw[2 * j + 1]);
+              acc[c] = __fmaf_rn(a, cc[j], -__fmul_rn(b, sc[j]));
+              acc[c + 1] = __fmaf_rn(a, sc[j], __fmul_rn(b, cc[j]));
+            }
+          }
+        }
+      }
       if (row < p.M) {
 #pragma unroll
         for (int c = 0; c < 64; c += 8) {
@@ -342,7 +405,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           if (n >= p.N) break;
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = __fadd_rn(acc[c + e], n + e < p.N ? __ldg(p.bias + n + e) : 0.0f);
+          for (int e = 0; e < 8; ++e)
+            y[e] = kQkv ? acc[c + e] : __fadd_rn(acc[c + e], n + e < p.N ? __ldg(p.bias + n + e) : 0.0f);
           if (n + 8 <= p.N && (p.N & 7) == 0) {
             if constexpr (kF32Out) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + static_cast<size_t>(row) * p.N + n);
@@ -393,7 +457,7 @@ teardown:
 }  // namespace
 
 cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* lora_act, int M,
-                             void* Y, int out_dtype, cudaStream_t s) {
+                             void* Y, int out_dtype, const svdq_qkv_prologue* pro, cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N;
   const int m_pad = static_cast<int>(m_pad_of(M));
   CUtensorMap tm_ap, tm_la;
@@ -420,9 +484,17 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   p.m_pad = m_pad;
   p.n_lora = w->rank_pad / 32;
   p.n_pad = w->n_pad;
+  p.norm_q = pro ? pro->norm_q : nullptr;
+  p.norm_k = pro ? pro->norm_k : nullptr;
+  p.rope_cos = pro ? pro->rope_cos : nullptr;
+  p.rope_sin = pro ? pro->rope_sin : nullptr;
+  p.eps = pro ? pro->eps : 0.0f;
+  p.qk_cols = pro ? 2 * pro->heads * pro->head_dim : 0;
   const int tiles = ((M + kTileM - 1) / kTileM) * ((N + kTileN - 1) / kTileN);
   const int grid = std::min(tiles, num_sms(w->device));
-  auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_int4_kernel<true> : gemm_int4_kernel<false>;
+  const bool f32 = out_dtype == SVDQ_OUT_F32;
+  auto kern = pro ? (f32 ? gemm_int4_kernel<true, true> : gemm_int4_kernel<false, true>)
+                  : (f32 ? gemm_int4_kernel<true, false> : gemm_int4_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kI4Smem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kI4Threads, kI4Smem, s>>>(tm_ap, w->tm_qw8, tm_la, w->tm_l2, p);

@@ -25,6 +25,17 @@
 // The lora-up shares the accumulator with the 4-bit product because
 // lora_act arrives pre-divided by g_x g_w.
 //
+// QKV variant (the FLUX to_qkv module of Nunchaku 4-bit in Diffusers,
+// "Quantisierung von Modellen mit strukturellen Umschreibungen": one fused
+// operator for the QKV projection, the Q/K normalisation and the rotary
+// embedding): Y = [Q | K | V] with sections of 256-column multiples, so a
+// tile is all Q, all K or all V.  In Q and K tiles the epilogue normalises
+// every 128-column head by its RMS (the head spans the 64 columns of two
+// warps of the same lane quarter, which add their sums of squares through
+// shared memory), scales by the per-dimension weight and turns the pairs
+// (2i, 2i+1) by the row's rotary angle, all in fp32 before the one
+// rounding to the output type.
+//
 // TMEM columns (same in both CTAs): [0, 256) accumulator (this CTA's 128
 // rows), then one scale slot of 48 columns per ring stage: 16 columns of A
 // scales (this CTA's rows) and 32 of B scales (all 256 columns; each CTA
@@ -61,7 +72,8 @@ constexpr int kStagingPerWarp = 2048;
 constexpr int kStagingOff = kStages * kStageBytes;
 constexpr int kBiasOff = kStagingOff + kEpiWarps * kStagingPerWarp;  // 2 x 256 floats
 constexpr int kBarOff = kBiasOff + 2 * BN * 4;
-constexpr size_t kSmemBytes = kBarOff + 256 /*barriers*/ + 1024 /*align*/;
+constexpr int kRedOff = kBarOff + 256;                     // QKV: one float per row of a head pair
+constexpr size_t kSmemBytes = kRedOff + 4 * 2 * 32 * 4 + 1024 /*align*/;
 
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -80,9 +92,16 @@ struct GemmParams {
   int M, N, K, n_lora;
   float gxgw;
   int tma_store;  // Y rows are whole multiples of 16 bytes: store through tm_y
+  // QKV attention prologue (the kQkv variant only)
+  const float* norm_q;
+  const float* norm_k;
+  const float* rope_cos;  // 64 x M, frequency-major
+  const float* rope_sin;
+  float eps;
+  int qk_cols;  // columns of Q and K (2 * heads * 128); K starts at qk_cols / 2
 };
 
-template <bool kF32Out>
+template <bool kF32Out, bool kQkv>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
@@ -91,6 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + kBiasOff);
+  float* red_s = reinterpret_cast<float*>(smem + kRedOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
@@ -269,6 +289,72 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       const int row = m0 + quarter * 32 + lane;
       const float* bb = bias_t + part * kColsPerWarp;
+      if constexpr (kQkv) {
+        // y = acc * RN32(g_x g_w) + b in place, then in Q / K tiles the
+        // head's RMS normalisation and rotary embedding (n0 is CTA-uniform,
+        // so every epilogue warp takes the same barriers)
+#pragma unroll
+        for (int c = 0; c < kColsPerWarp; ++c)
+          v[c] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(v[c]), p.gxgw), bb[c]));
+        if (n0 < p.qk_cols) {
+          const int hcol = (part & 1) * kColsPerWarp;  // first column of this half within its head
+          // rotary tables are frequency-major (pair i of token m at i * M + m):
+          // the warp's 32 rows of one frequency are one line.  The first
+          // group of four pairs is requested before the sum exchange, so
+          // that its L2 latency overlaps the barriers.
+          const bool in_rows = row < p.M;
+          const size_t trow = static_cast<size_t>(hcol / 2) * p.M + (in_rows ? row : 0);
+          const float* ct = p.rope_cos + trow;
+          const float* st = p.rope_sin + trow;
+          float c0[4], s0[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            c0[j] = in_rows ? __ldg(ct + static_cast<size_t>(j) * p.M) : 1.0f;
+            s0[j] = in_rows ? __ldg(st + static_cast<size_t>(j) * p.M) : 0.0f;
+          }
+          float ss = 0.0f;
+#pragma unroll
+          for (int c = 0; c < kColsPerWarp; ++c) ss = __fmaf_rn(__uint_as_float(v[c]), __uint_as_float(v[c]), ss);
+          // the head = parts (2h, 2h+1) of this quarter: the odd half posts
+          // its sum, the even half adds it to its own (even half first) and
+          // posts the head's total, which both then read.  The slot is next
+          // written after the next tile's first barrier, which every reader
+          // of this tile has passed.
+          float* slot = red_s + (quarter * 2 + (part >> 1)) * 32 + lane;
+          if (part & 1) *slot = ss;
+          named_bar_sync(3, 32 * kEpiWarps);
+          if (!(part & 1)) *slot = __fadd_rn(ss, *slot);
+          named_bar_sync(3, 32 * kEpiWarps);
+          const float r = rsqrtf(__fmaf_rn(*slot, 1.0f / 128.0f, p.eps));
+          const float4* wn = reinterpret_cast<const float4*>((n0 < p.qk_cols / 2 ? p.norm_q : p.norm_k) + hcol);
+#pragma unroll
+          for (int q4 = 0; q4 < kColsPerWarp / 8; ++q4) {  // four pairs per step
+            float cc[4], sc[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              cc[j] = q4 == 0 ? c0[j] : (in_rows ? __ldg(ct + static_cast<size_t>(4 * q4 + j) * p.M) : 1.0f);
+              sc[j] = q4 == 0 ? s0[j] : (in_rows ? __ldg(st + static_cast<size_t>(4 * q4 + j) * p.M) : 0.0f);
+            }
+            const float4 w0 = __ldg(wn + 2 * q4), w1 = __ldg(wn + 2 * q4 + 1);
+            // the head's scale folded into the weights: (y r) w = y (r w)
+            const float rw[8] = {__fmul_rn(r, w0.x), __fmul_rn(r, w0.y), __fmul_rn(r, w0.z), __fmul_rn(r, w0.w),
+                                 __fmul_rn(r, w1.x), __fmul_rn(r, w1.y), __fmul_rn(r, w1.z), __fmul_rn(r, w1.w)};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int c = 8 * q4 + 2 * j;
+              const float a = __fmul_rn(__uint_as_float(v[c]), rw[2 * j]);
+              const float b = __fmul_rn(__uint_as_float(v[c + 1]), rw[2 * j + 1]);
+              v[c] = __float_as_uint(__fmaf_rn(a, cc[j], -__fmul_rn(b, sc[j])));
+              v[c + 1] = __float_as_uint(__fmaf_rn(a, sc[j], __fmul_rn(b, cc[j])));
+            }
+          }
+        }
+      }
+      // the value stored for column `col` of the warp's 64
+      auto yv = [&](int col) -> float {
+        if constexpr (kQkv) return __uint_as_float(v[col]);
+        else return __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
+      };
       if (p.tma_store) {
         // y rows into a 64-byte-wide swizzled box (32 rows; row r's 16-byte
         // unit u at r * 64 + ((u ^ ((r >> 1) & 3)) << 4)), then a TMA store
@@ -282,11 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kColsPerBox; j += 4) {
             const int col = pass * kColsPerBox + j;  // within the warp's columns
-            const uint32_t* a = &v[col];
-            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(a[0]), p.gxgw), bb[col]);
-            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(a[1]), p.gxgw), bb[col + 1]);
-            const float y2 = __fadd_rn(__fmul_rn(__uint_as_float(a[2]), p.gxgw), bb[col + 2]);
-            const float y3 = __fadd_rn(__fmul_rn(__uint_as_float(a[3]), p.gxgw), bb[col + 3]);
+            const float y0 = yv(col), y1 = yv(col + 1), y2 = yv(col + 2), y3 = yv(col + 3);
             const int byte = j * (kF32Out ? 4 : 2);  // within the box's 64-byte row
             uint8_t* line = stg + lane * 64;
             const int unit = (byte >> 4) ^ ((lane >> 1) & 3);
@@ -311,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int col = 0; col < kColsPerWarp; ++col) {
           const int n = n0 + part * kColsPerWarp + col;
           if (n < p.N) {
-            const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
+            const float y = yv(col);
             if constexpr (kF32Out)
               static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
             else
@@ -349,7 +431,8 @@ teardown:
 }  // namespace
 
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
-                              const float* lora_act, int M, void* Y, int out_dtype, cudaStream_t s) {
+                              const float* lora_act, int M, void* Y, int out_dtype, const svdq_qkv_prologue* pro,
+                              cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N;
   const int64_t m_pad = m_pad_of(M);
   CUtensorMap tm_a, tm_sfa, tm_la;
@@ -374,6 +457,12 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   p.K = K;
   p.n_lora = w->rank_pad / 32;
   p.gxgw = g_x * w->g_w;  // RN32(g_x * g_w)
+  p.norm_q = pro ? pro->norm_q : nullptr;
+  p.norm_k = pro ? pro->norm_k : nullptr;
+  p.rope_cos = pro ? pro->rope_cos : nullptr;
+  p.rope_sin = pro ? pro->rope_sin : nullptr;
+  p.eps = pro ? pro->eps : 0.0f;
+  p.qk_cols = pro ? 2 * pro->heads * pro->head_dim : 0;
   // Y through TMA stores when its rows are whole multiples of 16 bytes
   const bool f32 = out_dtype == SVDQ_OUT_F32;
   const uint64_t row_bytes = static_cast<uint64_t>(N) * (f32 ? 4 : 2);
@@ -383,7 +472,8 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
                                        N, M, row_bytes, f32 ? 16 : 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int pairs = std::min(tiles, num_sms(w->device) / 2);
-  auto kern = out_dtype == SVDQ_OUT_F32 ? gemm_nvfp4_kernel<true> : gemm_nvfp4_kernel<false>;
+  auto kern = pro ? (f32 ? gemm_nvfp4_kernel<true, true> : gemm_nvfp4_kernel<false, true>)
+                  : (f32 ? gemm_nvfp4_kernel<true, false> : gemm_nvfp4_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

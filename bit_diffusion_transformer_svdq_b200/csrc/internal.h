@@ -76,10 +76,12 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
 cudaError_t launch_act_global_scale(const svdq_weights* w, const uint16_t* X, int M, float* g_x, cudaStream_t s);
 cudaError_t launch_quantize(const svdq_weights* w, const uint16_t* X, int M, float g_x, uint8_t* qx, void* sx,
                             float* lora_act, cudaStream_t s);
+// `pro` (may be null): the QKV attention prologue applied in the epilogue
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
-                              const float* lora_act, int M, void* Y, int out_dtype, cudaStream_t s);
+                              const float* lora_act, int M, void* Y, int out_dtype, const svdq_qkv_prologue* pro,
+                              cudaStream_t s);
 cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* lora_act, int M,
-                             void* Y, int out_dtype, cudaStream_t s);
+                             void* Y, int out_dtype, const svdq_qkv_prologue* pro, cudaStream_t s);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
 // link-time dependency on libcuda).  2-D, row-major, `inner` elements per

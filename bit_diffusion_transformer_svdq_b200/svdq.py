@@ -51,6 +51,22 @@ class WeightsView(ctypes.Structure):
                 ("inv_lambda", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
 
 
+class QkvPrologue(ctypes.Structure):
+    """svdq_qkv_prologue: the attention prologue of a fused QKV projection
+    (per-head RMS normalisation of Q and K with weights norm_q / norm_k,
+    rotary embedding with cos / sin tables stored frequency-major,
+    head_dim/2 x M: entry (i, m) for pair i of token m)."""
+    _fields_ = [("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("norm_q", ctypes.c_void_p), ("norm_k", ctypes.c_void_p), ("rope_cos", ctypes.c_void_p),
+                ("rope_sin", ctypes.c_void_p)]
+
+
+def make_qkv_prologue(heads: int, norm_q, norm_k, rope_cos, rope_sin, eps: float = 1e-6,
+                      head_dim: int = 128) -> QkvPrologue:
+    """The caller keeps the four device tensors alive while the struct is used."""
+    return QkvPrologue(heads, head_dim, float(eps), _ptr(norm_q), _ptr(norm_k), _ptr(rope_cos), _ptr(rope_sin))
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -69,8 +85,10 @@ _SIGS = {
     "svdq_act_scale_bytes": (_Z, [_P, _I]),
     "svdq_quantize_act_lora_down": (_I, [_P, _P, _I, _F, _P, _P, _P, _P]),
     "svdq_w4a4_gemm_lora_up": (_I, [_P, _P, _P, _F, _P, _I, _P, _I, _P]),
+    "svdq_w4a4_gemm_lora_up_qkv": (_I, [_P, _P, _P, _F, _P, _I, ctypes.POINTER(QkvPrologue), _P, _I, _P]),
     "svdq_workspace_bytes": (_Z, [_P, _I]),
     "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
+    "svdq_linear_forward_qkv": (_I, [_P, _P, _I, _F, ctypes.POINTER(QkvPrologue), _P, _I, _P, _Z, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _P, _I, _F, _P, _I, _P]),
     "svdq_device_status": (_I, [_P, _P]),
     "svdq_selftest_bounded_wait": (_I, [_P]),
@@ -195,6 +213,20 @@ def svdq_w4a4_gemm_lora_up(w: Weights, qx, sx, g_x: float, lora_act, M: int, Y, 
                            stream=None) -> None:
     _check(load_library().svdq_w4a4_gemm_lora_up(w.handle, _ptr(qx), _ptr(sx), float(g_x), _ptr(lora_act), M, _ptr(Y),
                                                  out_dtype, _stream(stream)), "svdq_w4a4_gemm_lora_up")
+
+
+def svdq_w4a4_gemm_lora_up_qkv(w: Weights, qx, sx, g_x: float, lora_act, M: int, pro: QkvPrologue, Y,
+                               out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    _check(load_library().svdq_w4a4_gemm_lora_up_qkv(w.handle, _ptr(qx), _ptr(sx), float(g_x), _ptr(lora_act), M,
+                                                     ctypes.byref(pro), _ptr(Y), out_dtype, _stream(stream)),
+           "svdq_w4a4_gemm_lora_up_qkv")
+
+
+def svdq_linear_forward_qkv(w: Weights, X, M: int, g_x: float, pro: QkvPrologue, Y, workspace, ws_bytes: int,
+                            out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    _check(load_library().svdq_linear_forward_qkv(w.handle, _ptr(X), M, float(g_x), ctypes.byref(pro), _ptr(Y),
+                                                  out_dtype, _ptr(workspace), ws_bytes, _stream(stream)),
+           "svdq_linear_forward_qkv")
 
 
 def svdq_linear_forward(w: Weights, X, M: int, g_x: float, Y, workspace, ws_bytes: int,

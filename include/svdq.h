@@ -194,6 +194,41 @@ SVDQ_API svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const ui
 SVDQ_API svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
                                    const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream);
 
+/* Attention prologue fused into the epilogue of a QKV projection.  The
+ * pages ("Quantisierung von Modellen mit strukturellen Umschreibungen",
+ * Nunchaku 4-bit in Diffusers) describe the FLUX to_qkv module: one
+ * quantised projection whose fused operator also applies the Q/K
+ * normalisation and the rotary embedding.  With Y = [Q | K | V] (each
+ * heads * head_dim columns) the epilogue stores
+ *     Q' = rope(rmsnorm(Q) * norm_q),  K' = rope(rmsnorm(K) * norm_k),  V
+ * where, per row and head, rmsnorm(q)[d] = q[d] / sqrt(mean_d(q^2) + eps)
+ * and rope turns the pairs (2i, 2i+1) of every head by the row's angle:
+ * (a, b) -> (a cos[m,i] - b sin[m,i], a sin[m,i] + b cos[m,i]).  The values
+ * normalised are the layer outputs before rounding (accumulator, lora-up
+ * and bias in fp32); the result is rounded once to the output dtype.
+ * Limits: head_dim == 128; the layer's N == 3 * heads * 128 with heads
+ * even; eps > 0.  All pointers [device], 16-byte aligned:
+ *   norm_q, norm_k   head_dim fp32 weights,
+ *   rope_cos, rope_sin   head_dim/2 x M fp32, frequency-major: the value
+ *                    for pair i of token m at [i * M + m] (32 consecutive
+ *                    tokens of one frequency are one 128-byte line, which
+ *                    is what the epilogue, one thread per token, reads). */
+typedef struct svdq_qkv_prologue {
+  int32_t heads;
+  int32_t head_dim;
+  float eps;
+  const float* norm_q;
+  const float* norm_k;
+  const float* rope_cos;
+  const float* rope_sin;
+} svdq_qkv_prologue;
+
+/* svdq_w4a4_gemm_lora_up with the QKV attention prologue above applied in
+ * its epilogue (NVFP4 and INT4).  Same arguments plus `pro` [host]. */
+SVDQ_API svdq_status svdq_w4a4_gemm_lora_up_qkv(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
+                                       const float* lora_act, int32_t M, const svdq_qkv_prologue* pro, void* Y,
+                                       int32_t out_dtype, void* stream);
+
 /* Workspace bytes of svdq_linear_forward for M rows (qx, sx, lora_act). */
 SVDQ_API size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M);
 
@@ -202,6 +237,11 @@ SVDQ_API size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M);
  * svdq_workspace_bytes(w, M), 1024-byte aligned). */
 SVDQ_API svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
                                 int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* svdq_linear_forward whose GEMM is svdq_w4a4_gemm_lora_up_qkv. */
+SVDQ_API svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
+                                    const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace,
+                                    size_t ws_bytes, void* stream);
 
 /* The layer forward without a caller-provided workspace.  No counterpart
  * in the pages: this exists for callers that cannot allocate device memory

@@ -28,6 +28,7 @@ __all__ = [
     "make_layer",
     "bf16_bits_from_f32",
     "f32_from_bf16_bits",
+    "qkv_prologue_inputs",
 ]
 
 
@@ -155,3 +156,16 @@ def make_layer(shape: LayerShape | str, seed: int, **overrides) -> LayerInputs:
 def stack_seed(block: int, layer: int) -> int:
     """Per-linear seed of the 57-block stack (4 linears per block)."""
     return 5000 + 4 * block + layer
+
+
+def qkv_prologue_inputs(M: int, head_dim: int, seed: int):
+    """Inputs of the fused QKV attention prologue: per-dimension RMS-norm
+    weights for Q and K (fp32, uniform in [0.5, 1.5], like trained
+    QK-norm scales around 1) and per-token rotary tables (fp32 cosines and
+    sines of angles drawn uniformly in [-pi, pi), M x head_dim/2), drawn
+    from (seed, M, head_dim)."""
+    rng = np.random.default_rng([seed, M, head_dim, 7])
+    norm_q = rng.uniform(0.5, 1.5, head_dim).astype(np.float32)
+    norm_k = rng.uniform(0.5, 1.5, head_dim).astype(np.float32)
+    ang = rng.uniform(-math.pi, math.pi, (M, head_dim // 2))
+    return norm_q, norm_k, np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)

@@ -50,10 +50,15 @@ def test_weights_bytes_validates_the_descriptor(svdq):
 
 
 def test_null_arguments_rejected_before_any_cuda_call(svdq):
+    import ctypes
     lib = svdq.load_library()
     assert lib.svdq_quantize_act_lora_down(None, None, 4, 1.0, None, None, None, None) == 1
     assert lib.svdq_w4a4_gemm_lora_up(None, None, None, 1.0, None, 4, None, 0, None) == 1
     assert lib.svdq_linear_forward(None, None, 4, 1.0, None, 0, None, 0, None) == 1
+    pro = svdq.QkvPrologue()
+    assert lib.svdq_w4a4_gemm_lora_up_qkv(None, None, None, 1.0, None, 4, ctypes.byref(pro), None, 0, None) == 1
+    assert lib.svdq_w4a4_gemm_lora_up_qkv(None, None, None, 1.0, None, 4, None, None, 0, None) == 1
+    assert lib.svdq_linear_forward_qkv(None, None, 4, 1.0, ctypes.byref(pro), None, 0, None, 0, None) == 1
     import ctypes
     out = ctypes.c_void_p()
     d = svdq.make_desc(256, 256, 16)

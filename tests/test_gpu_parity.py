@@ -312,3 +312,74 @@ def test_argument_errors(svdq):
     svdq.svdq_linear_forward(w, X, 0, float(ol.gx), Y, ws, ws.numel())  # M = 0 is a no-op
     bad = svdq.make_desc(100, 256, 16)
     assert svdq.svdq_weights_bytes(bad) == 0
+
+
+# ------------------------------------------------ fused QKV attention prologue
+# (heads, workload, overrides): N = 3 * heads * 128; ragged M, several tiles
+QKV_CASES = [
+    ("h2_ragged", 2, "qkv", dict(M=300, K=512, N=768)),
+    ("h4_rank16", 4, "qkv", dict(M=129, K=256, N=1536, rank=16)),
+    ("h2_rank0", 2, "stack_qkv", dict(M=64, K=320, N=768, rank=0)),
+]
+
+
+def _qkv_case(svdq, li, ol, heads, precision, out_dtype, through_forward=True):
+    from oracle import qkv as A
+    w = T.gpu_prepare(svdq, li, ol, precision)
+    M, N = li.shape.M, li.shape.N
+    nq, nk, cs, sn = synth.qkv_prologue_inputs(M, 128, 23)
+    # the library takes the tables frequency-major (head_dim/2 x M)
+    dq, dk, dc, ds = T.dev_f32(nq), T.dev_f32(nk), T.dev_f32(cs.T.copy()), T.dev_f32(sn.T.copy())
+    eps = 1e-6
+    pro = svdq.make_qkv_prologue(heads, dq, dk, dc, ds, eps)
+    X = T.dev_u16(li.x_bits)
+    Y = torch.empty((M, N), dtype=torch.float32 if out_dtype == 1 else torch.bfloat16, device="cuda")
+    gx = float(ol.gx)
+    if through_forward:
+        ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
+        svdq.svdq_linear_forward_qkv(w, X, M, gx, pro, Y, ws, ws.numel(), out_dtype)
+    else:
+        _, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, gx)
+        svdq.svdq_w4a4_gemm_lora_up_qkv(w, qx, sx, gx, la, M, pro, Y, out_dtype)
+    assert svdq.svdq_device_status(w) == 0
+    y = Y.float().cpu().numpy()
+    plain = V.forward(li.x, ol.prep, ol.gx if precision == "nvfp4" else None)
+    ref = A.qkv_prologue(plain, heads, 128, nq, nk, cs, sn, eps)
+    return y, ref
+
+
+@pytest.mark.parametrize("precision", ["nvfp4", "int4"])
+@pytest.mark.parametrize("out_dtype", [1, 0], ids=["f32", "bf16"])
+@pytest.mark.parametrize("name,heads,wl,over", QKV_CASES, ids=[c[0] for c in QKV_CASES])
+def test_qkv_prologue_parity(svdq, name, heads, wl, over, out_dtype, precision):
+    li = _layer(wl, over)
+    ol = T.oracle_layer(li, precision=precision)
+    y, ref = _qkv_case(svdq, li, ol, heads, precision, out_dtype, through_forward=(name != "h4_rank16"))
+    w = heads * 128
+    for sec in range(3):  # Q, K (normalised, unit scale) and V (the layer's own scale) separately
+        _assert_y(y[:, sec * w:(sec + 1) * w], ref[:, sec * w:(sec + 1) * w], out_dtype)
+
+
+def test_qkv_prologue_argument_errors(svdq):
+    li = _layer("qkv", dict(M=64, K=256, N=768))
+    ol = T.oracle_layer(li, precision="nvfp4")
+    w = T.gpu_prepare(svdq, li, ol, "nvfp4")
+    M = 64
+    X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
+    t = torch.ones(M * 64 + 4, dtype=torch.float32, device="cuda")
+    Y = torch.empty((M, 768), dtype=torch.bfloat16, device="cuda")
+    lib = svdq.load_library()
+    import ctypes
+
+    def call(pro):
+        return lib.svdq_w4a4_gemm_lora_up_qkv(w.handle, qx.data_ptr(), sx.data_ptr(), float(ol.gx), la.data_ptr(), M,
+                                              ctypes.byref(pro), Y.data_ptr(), 0, None)
+
+    good = svdq.make_qkv_prologue(2, t, t, t, t, 1e-6)
+    assert call(good) == 0
+    torch.cuda.synchronize()
+    assert call(svdq.make_qkv_prologue(3, t, t, t, t, 1e-6)) == 2          # N != 3 * heads * 128 (and odd)
+    assert call(svdq.make_qkv_prologue(2, t, t, t, t, 1e-6, head_dim=64)) == 2
+    assert call(svdq.make_qkv_prologue(2, t, t, t, t, 0.0)) == 1          # eps must be > 0
+    assert call(svdq.make_qkv_prologue(2, None, t, t, t, 1e-6)) == 1
+    assert call(svdq.make_qkv_prologue(2, t, t, t[1:], t, 1e-6)) == 3     # rope_cos not 16-byte aligned
