@@ -131,3 +131,40 @@ def test_stack_block_through_forward(svdq):
         assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F, name
         half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
         assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp), name
+
+
+def test_full_size_qkv_prologue(svdq):
+    """The fused QKV projection (M=4608, K=3072, N=9216 = 3 x 24 heads x
+    128, rank 32, NVFP4) with the attention prologue in the GEMM epilogue:
+    sampled rows of Q', K', V against the oracle's prologue applied to the
+    fp64 layer output."""
+    from oracle import qkv as A
+    li = synth.make_layer("qkv", 2)
+    M, K, N = li.shape.M, li.shape.K, li.shape.N
+    heads = N // 384
+    ol = T.oracle_layer(li)
+    w = T.gpu_prepare(svdq, li, ol)
+    X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
+    nq, nk, cs, sn = synth.qkv_prologue_inputs(M, 128, 29)
+    dq, dk, dc, ds = T.dev_f32(nq), T.dev_f32(nk), T.dev_f32(cs.T.copy()), T.dev_f32(sn.T.copy())
+    pro = svdq.make_qkv_prologue(heads, dq, dk, dc, ds, 1e-6)
+    rows = np.sort(np.random.default_rng(9).choice(M, SAMPLE_ROWS, replace=False))
+    act = V.quantize_activations(li.x[rows], ol.prep, ol.gx)
+    ref = A.qkv_prologue(V.forward_from_codes(act, ol.prep, ol.gx), heads, 128, nq, nk, cs[rows], sn[rows], 1e-6)
+    wd = heads * 128
+    for out_dtype in (1, 0):
+        Y = torch.empty((M, N), dtype=torch.float32 if out_dtype else torch.bfloat16, device="cuda")
+        svdq.svdq_w4a4_gemm_lora_up_qkv(w, qx, sx, float(ol.gx), la, M, pro, Y, out_dtype)
+        torch.cuda.synchronize()
+        y = Y.float().cpu().numpy()[rows].astype(np.float64)
+        for sec in range(3):
+            r_ = ref[:, sec * wd:(sec + 1) * wd]
+            d = y[:, sec * wd:(sec + 1) * wd] - r_
+            rms = np.sqrt(np.mean(r_ ** 2))
+            assert np.linalg.norm(d) / np.linalg.norm(r_) <= REL_F
+            if out_dtype:
+                assert np.abs(d).max() <= MAX_ABS * rms
+            else:
+                half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(r_), 1e-30))) - 8)
+                assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
+    assert svdq.svdq_device_status(w) == 0
