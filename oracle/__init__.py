@@ -31,5 +31,6 @@ Modules:
              with lora-down, and the fp64 forward
   qkv      - the attention prologue of the fused QKV projection (per-head
              RMS normalisation of Q and K, rotary embedding)
+  awq      - the awq_w4a16 layer (INT4 group-64 weights, 16-bit activations)
 """
-from . import formats, qkv, quant, svd, svdq  # noqa: F401
+from . import awq, formats, qkv, quant, svd, svdq  # noqa: F401
