@@ -401,6 +401,71 @@ def run_stack(args, rank, world, local_rank):
             "gpu_launches": 2 * len(layers) * args.steps, "clocks": clocks}), flush=True)
 
 
+def run_awq(args, rank, world, local_rank):
+    """The awq_w4a16 family on its FLUX workload: a double block's adaLN
+    modulation (3072 -> 6 x 3072) for a batch of `--batch` images, seeded
+    random weights and activation-aware channel scales, L2 read-flushed
+    before every step.  Memory-bound: the roofline is the HBM copy rate
+    against the weight codes + scales + X + Y bytes."""
+    import torch
+    import synth
+    from bit_diffusion_transformer_svdq_b200 import svdq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    svdq.load_library()
+    stream = torch.cuda.current_stream()
+    li = synth.make_layer("awq", SEED, M=args.batch)
+    M, K, N = li.shape.M, li.shape.K, li.shape.N
+    W = torch.from_numpy(li.w).to(dev)
+    alpha = torch.from_numpy(synth.awq_alpha(K, SEED)).to(dev)
+    b = torch.from_numpy(li.bias_bits.view(np.int16)).to(dev)
+    w = svdq.prepare_layer(W, alpha, None, None, b, 0, svdq.SVDQ_AWQ_W4A16)
+    del W
+    X = torch.from_numpy(li.x_bits.view(np.int16)).to(dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        flush.sum()
+        svdq.svdq_awq_w4a16_forward(w, X, M, Y, svdq.SVDQ_OUT_BF16, stream)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler.start()
+    time.sleep(0.1)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ev = []
+    for _ in range(args.steps):
+        flush.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        svdq.svdq_awq_w4a16_forward(w, X, M, Y, svdq.SVDQ_OUT_BF16, stream)
+        e1.record(stream)
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    _barrier(world)
+    clocks = sampler.stop(t_wall0, time.time())
+    assert svdq.svdq_device_status(w) == 0
+    t_ms = _allreduce_max(sum(a.elapsed_time(c) for a, c in ev) / len(ev), world, dev)
+    nbytes = N * K // 2 + (K // 64) * N * 2 + M * K * 2 + M * N * 2 + K * 4 + N * 4
+    peaks, peak_kind = _peaks()
+    gbs = nbytes / (t_ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "awq_w4a16 modulation projection, GB/s of weight + activation traffic",
+            "value": world * gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4 weights x fp32 (bf16 activations)", "data": "synthetic",
+            "config": {"workload": f"awq adaLN modulation M={M} K={K} N={N} int4/64",
+                       "l2": "flushed (256 MiB read) before each step", "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "kernel": "awq_gemv_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": nbytes, "peak_source": f"{peak_kind} hbm_gbs"},
+            "gpu_launches": args.steps, "clocks": clocks}), flush=True)
+
+
 def _barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -425,8 +490,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=None, help="override M (smaller profiling cases only)")
-    ap.add_argument("--workload", default="qkv", choices=["qkv", "stack"],
-                    help="qkv: the single-layer bench line; stack: one denoising step of the block stack")
+    ap.add_argument("--workload", default="qkv", choices=["qkv", "stack", "awq"],
+                    help="qkv: the single-layer bench line; stack: one denoising step of the block stack; "
+                         "awq: the awq_w4a16 modulation projection")
+    ap.add_argument("--batch", type=int, default=1, help="rows of the awq workload (images)")
     ap.add_argument("--blocks", type=int, default=57, help="blocks of the stack workload")
     ap.add_argument("--qkv-prologue", action="store_true",
                     help="qkv workload: the GEMM also applies the QK-norm + rotary attention prologue")
@@ -448,9 +515,9 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    if args.workload == "stack":
+    if args.workload in ("stack", "awq"):
         try:
-            run_stack(args, rank, world, local_rank)
+            (run_stack if args.workload == "stack" else run_awq)(args, rank, world, local_rank)
         finally:
             if world > 1:
                 import torch.distributed as dist

@@ -38,6 +38,9 @@ svdq_status check_desc(const svdq_layer_desc* d) {
     if (d->group_size != 16) return SVDQ_ERR_INVALID_ARG;
   } else if (d->precision == SVDQ_INT4) {
     if (d->group_size != 64) return SVDQ_ERR_INVALID_ARG;
+  } else if (d->precision == SVDQ_AWQ_W4A16) {
+    if (d->group_size != 64) return SVDQ_ERR_INVALID_ARG;
+    if (d->rank != 0) return SVDQ_ERR_SHAPE;  // no low-rank branch in this family
   } else {
     return SVDQ_ERR_INVALID_ARG;
   }
@@ -112,7 +115,8 @@ WeightLayout weight_layout(const svdq_layer_desc& d) {
     off = static_cast<size_t>(round_up(static_cast<int64_t>(off + bytes), 1024));
     return at;
   };
-  L.qw = take(static_cast<size_t>(d.N) * d.K / 2);
+  const bool awq = d.precision == SVDQ_AWQ_W4A16;
+  L.qw = take(static_cast<size_t>(awq ? np : d.N) * d.K / 2);  // awq: GEMV tiles over n_pad rows
   L.sw_bytes = d.precision == SVDQ_NVFP4 ? nvfp4_scale_bytes(np, d.K) : int4_scale_bytes(np, d.K);
   L.sw = take(L.sw_bytes);
   L.l1s = take(static_cast<size_t>(rp) * d.K * 2);
@@ -276,7 +280,7 @@ svdq_status svdq_weights_get_view(const svdq_weights* w, svdq_weights_view* v) {
 }
 
 svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t* X, int32_t M, float* g_x, void* stream) {
-  if (!w || !X || !g_x) return SVDQ_ERR_INVALID_ARG;
+  if (!w || !X || !g_x || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M <= 0) return SVDQ_ERR_SHAPE;
   if (!aligned16(X) || (reinterpret_cast<uintptr_t>(g_x) & 3u)) return SVDQ_ERR_ALIGNMENT;
   int dev;
@@ -293,7 +297,7 @@ size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M) {
 
 svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, uint8_t* qx,
                                         void* sx, float* lora_act, void* stream) {
-  if (!w) return SVDQ_ERR_INVALID_ARG;
+  if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;  // 16-bit activations there
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!X || !qx || !sx || (w->rank_pad > 0 && !lora_act)) return SVDQ_ERR_INVALID_ARG;
@@ -310,7 +314,7 @@ namespace {
 // Shared by the GEMM entry points: argument checks, then the launch.
 svdq_status gemm_entry(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x, const float* lora_act,
                        int32_t M, const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* stream) {
-  if (!w) return SVDQ_ERR_INVALID_ARG;
+  if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!qx || !sx || !Y || (w->rank_pad > 0 && !lora_act)) return SVDQ_ERR_INVALID_ARG;
@@ -365,7 +369,7 @@ namespace {
 svdq_status forward_entry(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
                           const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace, size_t ws_bytes,
                           void* stream) {
-  if (!w) return SVDQ_ERR_INVALID_ARG;
+  if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!workspace) return SVDQ_ERR_INVALID_ARG;
@@ -392,6 +396,20 @@ svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, in
   const svdq_status st = check_qkv(w, pro);
   if (st != SVDQ_OK) return st;
   return forward_entry(w, X, M, g_x, pro, Y, out_dtype, workspace, ws_bytes, stream);
+}
+
+svdq_status svdq_awq_w4a16_forward(const svdq_weights* w, const uint16_t* X, int32_t M, void* Y, int32_t out_dtype,
+                                   void* stream) {
+  if (!w || w->desc.precision != SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0) return SVDQ_ERR_SHAPE;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (out_dtype != SVDQ_OUT_BF16 && out_dtype != SVDQ_OUT_F32) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Y)) return SVDQ_ERR_ALIGNMENT;
+  int dev;
+  svdq_status st = current_device(&dev);
+  if (st != SVDQ_OK) return st;
+  return from_cuda(launch_awq_gemv(w, X, M, Y, out_dtype, static_cast<cudaStream_t>(stream)));
 }
 
 svdq_status svdq_device_status(const svdq_weights* w, void* stream) {

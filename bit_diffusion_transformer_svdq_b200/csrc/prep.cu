@@ -78,7 +78,7 @@ template <bool kInt4>
 __global__ void quantize_weights_kernel(const float* __restrict__ W, const float* __restrict__ lam,
                                         const uint16_t* __restrict__ L1, const uint16_t* __restrict__ L2, int N,
                                         int K, int r, const float* __restrict__ g_w_ptr, int64_t n_pad,
-                                        uint8_t* __restrict__ qw, uint8_t* __restrict__ sw) {
+                                        uint8_t* __restrict__ qw, uint8_t* __restrict__ sw, int gemv_tiles) {
   const int groups = K / 16;
   const size_t total = static_cast<size_t>(N) * groups;
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -137,7 +137,14 @@ __global__ void quantize_weights_kernel(const float* __restrict__ W, const float
     }
     if (valid && (j & 3) == 0) reinterpret_cast<__half*>(sw)[static_cast<size_t>(j >> 2) * n_pad + n] = s_h;
   }
-  if (valid) *reinterpret_cast<uint2*>(qw + static_cast<size_t>(n) * (K / 2) + k0 / 2) = make_uint2(lo, hi);
+  if (valid) {
+    // row-major, or (awq_w4a16) the GEMV tiles: 16 bytes per 32 codes of a
+    // row, 32 rows of a chunk contiguous
+    const size_t off = gemv_tiles ? (static_cast<size_t>(n >> 5) * (K / 32) + (k0 >> 5)) * 512 + (n & 31) * 16 +
+                                        ((k0 >> 4) & 1) * 8
+                                  : static_cast<size_t>(n) * (K / 2) + k0 / 2;
+    *reinterpret_cast<uint2*>(qw + off) = make_uint2(lo, hi);
+  }
 }
 
 // INT4 working copies: unpacked codes (K permuted within 8-value blocks,
@@ -193,6 +200,7 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
                            const uint16_t* L2, const uint16_t* bias, cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N, r = w->desc.rank, rp = w->rank_pad;
   const bool int4 = w->desc.precision == SVDQ_INT4;
+  const bool awq = w->desc.precision == SVDQ_AWQ_W4A16;
   float* g_w_dev = reinterpret_cast<float*>(w->amax + 1);
   cudaError_t e;
   if ((e = cudaMemsetAsync(w->sw, 0, w->sw_bytes, s)) != cudaSuccess) return e;
@@ -201,15 +209,20 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
   inv_lambda_kernel<<<(K + 255) / 256, 256, 0, s>>>(lambda, K, w->inv_lambda);
   const size_t chunks = static_cast<size_t>(N) * (K / 16);
   const int sms = num_sms(w->device);
-  if (!int4) {
+  if (awq) {
+    // the tile layout covers n_pad rows: the rows past N keep zero codes
+    if ((e = cudaMemsetAsync(w->qw, 0, static_cast<size_t>(w->n_pad) * (K / 2), s)) != cudaSuccess) return e;
+    quantize_weights_kernel<true><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
+        W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw), 1);
+  } else if (!int4) {
     const int blocks = static_cast<int>(std::min<size_t>((chunks + 255) / 256, static_cast<size_t>(sms) * 16));
     residual_amax_kernel<<<std::max(blocks, 1), 256, 0, s>>>(W, lambda, L1, L2, N, K, r, w->amax);
     weight_scale_kernel<<<1, 1, 0, s>>>(w->amax, g_w_dev);
     quantize_weights_kernel<false><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
-        W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw));
+        W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw), 0);
   } else {
     quantize_weights_kernel<true><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
-        W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw));
+        W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw), 0);
     const size_t work = std::max(static_cast<size_t>(w->n_pad) * (K / 8), static_cast<size_t>(K / 64) * w->n_pad);
     int4_unpack_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(
         w->qw, static_cast<const __half*>(w->sw), N, K, w->n_pad, w->qw8, w->swp);

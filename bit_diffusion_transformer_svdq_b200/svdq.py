@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libsvdq.so")
 
 SVDQ_NVFP4 = 0
 SVDQ_INT4 = 1
+SVDQ_AWQ_W4A16 = 2
 SVDQ_OUT_BF16 = 0
 SVDQ_OUT_F32 = 1
 
@@ -90,6 +91,7 @@ _SIGS = {
     "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
     "svdq_linear_forward_qkv": (_I, [_P, _P, _I, _F, ctypes.POINTER(QkvPrologue), _P, _I, _P, _Z, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _P, _I, _F, _P, _I, _P]),
+    "svdq_awq_w4a16_forward": (_I, [_P, _P, _I, _P, _I, _P]),
     "svdq_device_status": (_I, [_P, _P]),
     "svdq_selftest_bounded_wait": (_I, [_P]),
 }
@@ -243,6 +245,13 @@ def svdq_linear_forward_noalloc(w: Weights, X, M: int, g_x: float, Y, out_dtype:
     on that scratch."""
     _check(load_library().svdq_linear_forward_noalloc(w.handle, _ptr(X), M, float(g_x), _ptr(Y), out_dtype,
                                                       _stream(stream)), "svdq_linear_forward_noalloc")
+
+
+def svdq_awq_w4a16_forward(w: Weights, X, M: int, Y, out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    """The awq_w4a16 layer: Y = X_hat dequant(q, s)^T + b for weights
+    prepared with precision SVDQ_AWQ_W4A16 (lambda = the AWQ channel scale)."""
+    _check(load_library().svdq_awq_w4a16_forward(w.handle, _ptr(X), M, _ptr(Y), out_dtype, _stream(stream)),
+           "svdq_awq_w4a16_forward")
 
 
 def svdq_device_status(w: Weights, stream=None) -> int:

@@ -65,8 +65,10 @@ typedef enum svdq_status {
 } svdq_status;
 
 typedef enum svdq_precision {
-  SVDQ_NVFP4 = 0, /* E2M1 codes, E4M3 scale per 16, fp32 tensor scale */
-  SVDQ_INT4 = 1   /* signed 4-bit codes, fp16 scale per 64 */
+  SVDQ_NVFP4 = 0,     /* E2M1 codes, E4M3 scale per 16, fp32 tensor scale */
+  SVDQ_INT4 = 1,      /* signed 4-bit codes, fp16 scale per 64 */
+  SVDQ_AWQ_W4A16 = 2  /* the awq_w4a16 family: INT4 group-64 weights, 16-bit
+                         activations (see svdq_awq_w4a16_forward) */
 } svdq_precision;
 
 typedef enum svdq_out_dtype {
@@ -74,7 +76,9 @@ typedef enum svdq_out_dtype {
   SVDQ_OUT_F32 = 1   /* parity/debug output: the same epilogue stored in fp32 */
 } svdq_out_dtype;
 
-/* One quantised linear layer (the svdq_w4a4 block of quantization_config). */
+/* One quantised linear layer (the svdq_w4a4 block of quantization_config;
+ * with precision SVDQ_AWQ_W4A16 the awq_w4a16 block: group_size 64,
+ * rank 0). */
 typedef struct svdq_layer_desc {
   int32_t K;          /* input features */
   int32_t N;          /* output features */
@@ -92,9 +96,15 @@ typedef struct svdq_weights svdq_weights;
  * All pointers are [device] and point into the caller's storage.
  *   qw        N x K/2 bytes, two codes per byte, even k in the low nibble.
  *             NVFP4: E2M1 nibbles (bit 3 = sign); INT4: two's complement.
+ *             AWQ_W4A16: two's complement in the GEMV tile layout: rows
+ *             padded to n_pad (zero codes), and the 16 bytes holding codes
+ *             32c .. 32c+31 of row n at
+ *                 ((n / 32) * (K / 32) + c) * 512 + (n % 32) * 16,
+ *             so that 32 consecutive rows of one 32-code chunk are 512
+ *             contiguous bytes.
  *   sw        NVFP4: E4M3 bytes in the tiled scale layout (below) with
  *             rows = N padded to a multiple of 256.
- *             INT4: fp16, group-major: sw[g * n_pad + n], g < K/64.
+ *             INT4 and AWQ_W4A16: fp16, group-major: sw[g * n_pad + n], g < K/64.
  *   l1s       rank_pad x K bf16: bf16(RN32(L1[t,k] * inv_lambda[k])),
  *             rows t >= rank are zero.
  *   l2        N x rank_pad fp32 copy of L2 (exact), columns t >= rank zero.
@@ -263,6 +273,22 @@ SVDQ_API svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16
  * (other streams, other host threads) race on it. */
 SVDQ_API svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
                                                  void* Y, int32_t out_dtype, void* stream);
+
+/* The awq_w4a16 layer (Nunchaku 4-bit in Diffusers: the second kernel
+ * family, 4-bit weights with 16-bit activations, for the memory-bound and
+ * precision-sensitive modulation projections such as FLUX adanorm_zero /
+ * adanorm_single; quantization_config "awq_w4a16": int4, group_size 64).
+ * Weights come from svdq_prepare_weights with precision SVDQ_AWQ_W4A16,
+ * rank 0, `lambda` = the activation-aware per-input-channel scale alpha
+ * (K fp32; ones when there is none): W_til = RN32(W * alpha) quantised by
+ * the INT4 group-64 rule of svdq_prepare_weights.  This call computes
+ *     Y = X_hat (s_h q)^T + b,   X_hat = RN32(X * RN32(1 / alpha)),
+ * with fp32 accumulation, stored as bf16 (RNE) or fp32 (out_dtype).
+ * X [device] M x K bf16 (M >= 0, typically the batch), Y [device] M x N.
+ * Memory-bound GEMV-shaped work on the CUDA cores; no workspace.  Returns
+ * SVDQ_ERR_INVALID_ARG for weights of another precision. */
+SVDQ_API svdq_status svdq_awq_w4a16_forward(const svdq_weights* w, const uint16_t* X, int32_t M, void* Y,
+                                   int32_t out_dtype, void* stream);
 
 /* Synchronises `stream` and returns (then clears) the status word that the
  * GEMM kernels of this weight set write when a bounded wait runs out:

@@ -85,6 +85,9 @@ WORKLOADS = {
     "stack_out": LayerShape("stack_out", 4608, 3072, 3072, 32, "nvfp4", 16, "outlier4x50", "gauss"),
     "stack_up": LayerShape("stack_up", 4608, 3072, 12288, 32, "nvfp4", 16, "outlier4x50", "gauss"),
     "stack_down": LayerShape("stack_down", 4608, 12288, 3072, 32, "nvfp4", 16, "outlier4x50", "gauss"),
+    # the awq_w4a16 family: a FLUX double block's adaLN modulation (conditioning
+    # vector after SiLU, 3072 -> 6 x 3072), one row per image
+    "awq": LayerShape("awq", 1, 3072, 18432, 0, "awq", 64, "silu", "gauss"),
 }
 
 STACK_BLOCKS = 57
@@ -112,6 +115,9 @@ def _draw_x(rng: np.random.Generator, M: int, K: int, dist: str) -> np.ndarray:
     if dist == "gelu1.5":
         v = rng.standard_normal((M, K), dtype=np.float32) * np.float32(1.5)
         return _gelu_tanh(v.astype(np.float64)).astype(np.float32)
+    if dist == "silu":  # SiLU of N(0, 1): the conditioning input of a modulation projection
+        v = rng.standard_normal((M, K)).astype(np.float64)
+        return (v / (1.0 + np.exp(-v))).astype(np.float32)
     if dist == "student3":
         return (0.5 * rng.standard_t(3.0, size=(M, K))).astype(np.float32)
     raise ValueError(dist)
@@ -169,3 +175,11 @@ def qkv_prologue_inputs(M: int, head_dim: int, seed: int):
     norm_k = rng.uniform(0.5, 1.5, head_dim).astype(np.float32)
     ang = rng.uniform(-math.pi, math.pi, (M, head_dim // 2))
     return norm_q, norm_k, np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def awq_alpha(K: int, seed: int) -> np.ndarray:
+    """An activation-aware per-input-channel scale for the awq_w4a16 layer:
+    positive fp32 factors exp(U(-0.5, 0.5)) (a calibration would put them
+    near 1), drawn from (seed, K)."""
+    rng = np.random.default_rng([seed, K, 11])
+    return np.exp(rng.uniform(-0.5, 0.5, K)).astype(np.float32)
