@@ -11,24 +11,29 @@
 //               activation codes (128 rows x 64 B, 64-byte swizzled) and the
 //               prepared int8 weight codes (128 rows x 128 B, 128-byte
 //               swizzled); per tile one stage of lora_act / L2 (fp32).
-//   warps 2-5   converters: one row each, unpack the packed activation codes
-//               into int8 in the 128-byte-swizzled layout of the MMA operand
-//               (same K permutation as the prepared weights).
+//   warps 2-3   converters: two rows per lane, unpack the packed activation
+//               codes into int8 in the 128-byte-swizzled layout of the MMA
+//               operand (same K permutation as the prepared weights).
 //   warp 1      TMEM owner and MMA issuer: per group two kind::i8 MMAs
 //               (K = 32) into one of four int32 accumulators (128 columns
 //               each), so the MMAs run up to three groups ahead of the
 //               scaling; per tile four kind::tf32 MMAs of the lora-up into
 //               the next accumulator, as one more "group" of scale 1.
-//   warps 6-13  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM lane
-//               quarter) and 64 columns; per group it reads the int32
-//               product and adds RN(P s_w) s_x to its fp32 accumulator.
-//               RN(P s_w) is one FMA on the bit pattern magic + P (exact for
-//               |P| < 2^22; a group's |P| is at most 64 * 8 * 8), no
-//               int-to-float conversion.  Finally y = acc + b is stored;
-//               the QKV variant first applies the attention prologue (per
-//               128-column head of Q and K: RMS normalisation, weight,
-//               rotary embedding), the two column halves of a row adding
-//               their sums of squares through shared memory.
+//   warps 4-19  epilogue: warp e = w - 4 owns rows 32 (e % 4) .. + 31 (its
+//               TMEM lane quarter) and columns 32 (e / 4) .. + 31; per group
+//               it reads its int32 products, frees the accumulator and adds
+//               RN(P s_w) s_x to its fp32 accumulator.  RN(P s_w) is one FMA
+//               on the bit pattern magic + P (exact for |P| < 2^22; a
+//               group's |P| is at most 64 * 8 * 8), no int-to-float
+//               conversion.  The producer bulk-copies each group's scales
+//               into a ring of eight shared-memory entries (released with
+//               one arrival per epilogue warp), so the 16 warps never wait
+//               for one another between groups.  Finally y = acc + b is
+//               stored; the QKV variant first applies the attention
+//               prologue (per 128-column head of Q and K: RMS
+//               normalisation, weight, rotary embedding), the four column
+//               slices of a row adding their sums of squares through shared
+//               memory.
 // The group rescale is CUDA-core work on every output element (three
 // operations per element per 64 K, against 64 MACs on the tensor core), so
 // this kernel is bound by it, not by the MMAs.
@@ -49,19 +54,24 @@ constexpr int kApBytes = kTileM * 64;    // packed activation codes of a stage: 
 constexpr int kA8Bytes = kTileM * 128;   // unpacked
 constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes
 constexpr int kI4StageBytes = kApBytes + kA8Bytes + kB8Bytes;  // 40 KB
-constexpr int kConvWarps = 4;
-constexpr int kI4EpiWarps = 8;  // 4 lane quarters x 2 column halves
+constexpr int kConvWarps = 2;  // each lane unpacks two rows (r, r + 64)
+constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
 constexpr int kI4Threads = 32 * (2 + kConvWarps + kI4EpiWarps);
 constexpr int kAccBufs = 4;  // int32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
 constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
-// Group scales reach the epilogue through a ring of kScaleSlots groups in
-// shared memory, each thread fetching its value kScaleAhead groups early
-// (one global load's latency is much longer than a group's work).
-constexpr int kScaleSlots = 8, kScaleAhead = 4;
-constexpr int kScaleOff = kI4Stages * kI4StageBytes;  // per slot: 128 float2 s_w pairs + 128 float s_x
-constexpr int kI4BarOff = kScaleOff + kScaleSlots * (kTileN * 8 + kTileM * 4);
-constexpr int kI4RedOff = kI4BarOff + 512;  // QKV: one float per row of a head (4 x 32)
-constexpr size_t kI4Smem = kI4RedOff + 4 * 32 * 4 + 1024 /*align*/;
+// Group scales reach the epilogue through a ring of kScaleSlots entries in
+// shared memory, filled by the producer with bulk copies: per entry the
+// tile's 128 (s_w, -magic s_w) pairs and its 128 fp16 s_x.
+constexpr int kScaleSlots = 8;
+constexpr int kScaleSlotBytes = kTileN * 8 + kTileM * 2;  // 1280
+constexpr int kScaleOff = kI4Stages * kI4StageBytes;
+// each epilogue warp's private copy of its current group's scales: 32
+// (s_w, -magic s_w) pairs and 32 s_x
+constexpr int kPrivOff = kScaleOff + kScaleSlots * kScaleSlotBytes;
+constexpr int kPrivBytes = 32 * 8 + 32 * 4;
+constexpr int kI4BarOff = kPrivOff + kI4EpiWarps * kPrivBytes;
+constexpr int kI4RedOff = kI4BarOff + 512;  // QKV: one float per row and column slice (16 x 32)
+constexpr size_t kI4Smem = kI4RedOff + kI4EpiWarps * 32 * 4 + 1024 /*align*/;
 static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 static_assert(kI4Smem <= 232448, "shared memory budget");
 
@@ -102,15 +112,15 @@ __global__ void __launch_bounds__(kI4Threads, 1)
                      const I4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float2* sc_sw = reinterpret_cast<float2*>(smem + kScaleOff);                          // [slots][128]
-  float* sc_sx = reinterpret_cast<float*>(smem + kScaleOff + kScaleSlots * kTileN * 8);  // [slots][128]
   float* red_s = reinterpret_cast<float*>(smem + kI4RedOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
-  uint64_t* conv = full + kI4Stages;      // activation codes unpacked (4 converter warps)
+  uint64_t* conv = full + kI4Stages;      // activation codes unpacked (one arrival per converter warp)
   uint64_t* empty = conv + kI4Stages;     // MMAs done with the stage
   uint64_t* acc_full = empty + kI4Stages;      // [kAccBufs]
-  uint64_t* acc_empty = acc_full + kAccBufs;   // [kAccBufs], 8 epilogue warps
-  uint64_t* drain = acc_empty + kAccBufs;
+  uint64_t* acc_empty = acc_full + kAccBufs;   // [kAccBufs], one arrival per epilogue warp
+  uint64_t* sc_full = acc_empty + kAccBufs;    // [kScaleSlots], bulk copies of a group's scales
+  uint64_t* sc_empty = sc_full + kScaleSlots;  // [kScaleSlots], one arrival per epilogue warp
+  uint64_t* drain = sc_empty + kScaleSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -132,6 +142,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kI4EpiWarps);
     }
+    for (int b = 0; b < kScaleSlots; ++b) {
+      mbar_init(&sc_full[b], 1);
+      mbar_init(&sc_empty[b], kI4EpiWarps);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -145,6 +159,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   uint32_t issued_mask = 0, issued_par = 0;
+  uint32_t sc_mask = 0, sc_par = 0;  // scale-ring entries issued (teardown drain)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (whole warp)
@@ -154,6 +169,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
     int stage = 0;
     uint32_t phase = 0;
+    uint32_t sc_count = 0;  // scale-ring entries issued so far
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
       for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
@@ -175,28 +191,51 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+        // the scales of this stage's groups, one ring entry per group (after
+        // the operands, so that a slow epilogue never holds the MMAs back)
+        if (kb < num_kb) {
+          const int ng = min(2, groups - 2 * kb);
+          for (int gi = 0; gi < ng; ++gi, ++sc_count) {
+            const uint32_t ss = sc_count % kScaleSlots;
+            const uint32_t sp = (sc_count / kScaleSlots) & 1;
+            if (!mbar_wait_warp(&sc_empty[ss], sp ^ 1, abort_flag)) goto teardown;
+            if (elect_one()) {
+              const int g = 2 * kb + gi;
+              uint8_t* dst = smem + kScaleOff + ss * kScaleSlotBytes;
+              mbar_arrive_expect_tx(&sc_full[ss], kScaleSlotBytes);
+              bulk_load(dst, p.swp + static_cast<size_t>(g) * p.n_pad + n0, kTileN * 8, &sc_full[ss]);
+              bulk_load(dst + kTileN * 8, p.sx + static_cast<size_t>(g) * p.m_pad + m0, kTileM * 2, &sc_full[ss]);
+            }
+            __syncwarp();
+            sc_mask |= 1u << ss;
+            sc_par = (sc_par & ~(1u << ss)) | (sp << ss);
+          }
+        }
       }
     }
   } else if (warp >= 2 && warp < 2 + kConvWarps) {
     // ------------------------------------------------------- converters
-    const int r = (warp - 2) * 32 + lane;  // row of the tile
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
         if (kb < num_kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) goto teardown;
-          const uint8_t* ap = smem + stage * kI4StageBytes + r * 64;
-          uint8_t* a8 = smem + stage * kI4StageBytes + kApBytes + r * 128;
-          uint4 in[4];
+#pragma unroll 1
+          for (int rr = 0; rr < kTileM / (32 * kConvWarps); ++rr) {
+            const int r = (rr * kConvWarps + warp - 2) * 32 + lane;  // row of the tile
+            const uint8_t* ap = smem + stage * kI4StageBytes + r * 64;
+            uint8_t* a8 = smem + stage * kI4StageBytes + kApBytes + r * 128;
+            uint4 in[4];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) in[j] = *reinterpret_cast<const uint4*>(ap + ((j ^ ((r >> 1) & 3)) << 4));
-          const uint32_t w[16] = {in[0].x, in[0].y, in[0].z, in[0].w, in[1].x, in[1].y, in[1].z, in[1].w,
-                                  in[2].x, in[2].y, in[2].z, in[2].w, in[3].x, in[3].y, in[3].z, in[3].w};
+            for (int j = 0; j < 4; ++j) in[j] = *reinterpret_cast<const uint4*>(ap + ((j ^ ((r >> 1) & 3)) << 4));
+            const uint32_t w[16] = {in[0].x, in[0].y, in[0].z, in[0].w, in[1].x, in[1].y, in[1].z, in[1].w,
+                                    in[2].x, in[2].y, in[2].z, in[2].w, in[3].x, in[3].y, in[3].z, in[3].w};
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) =
-                make_uint4(unpack_lo(w[2 * u]), unpack_hi(w[2 * u]), unpack_lo(w[2 * u + 1]), unpack_hi(w[2 * u + 1]));
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) =
+                  make_uint4(unpack_lo(w[2 * u]), unpack_hi(w[2 * u]), unpack_lo(w[2 * u + 1]), unpack_hi(w[2 * u + 1]));
+          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(&conv[stage]);
@@ -260,123 +299,103 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // warp w owns rows 32 (w % 4) .. + 31 (its TMEM lane quarter) and 64
-    // columns.  A group's 128 s_w pairs and 128 s_x reach it through a ring
-    // of kScaleSlots entries in shared memory, one value per thread and entry,
-    // fetched kScaleAhead entries early.  The ring runs over the CTA's whole
-    // stream of (tile, group) pairs, index t, slot t % kScaleSlots: a thread
-    // writes entry t + kScaleAhead only after passing barrier t - 1, when every
-    // reader of entry t - kScaleAhead (same slot) is done.
-    const int q4 = warp & 3;
-    const int ch = (warp - 2 - kConvWarps) >> 2;         // columns 64 ch .. + 63
-    const int et = (warp - 2 - kConvWarps) * 32 + lane;  // 0 .. 255: s_w pair (< 128) or s_x
-    const int r = 32 * q4 + lane;
+    // warp e = 0..15 owns rows 32 (e % 4) .. + 31 (its TMEM lane quarter)
+    // and columns 32 (e / 4) .. + 31.  Per group it reads its 32 int32
+    // products, frees the accumulator (one arrival per warp) and adds
+    // RN(P s_w) s_x to its fp32 accumulator in registers.  The group's
+    // scales come from the producer's ring (waited for per warp, released
+    // with one arrival per warp): the warps never wait for one another.
+    const int e = warp - 2 - kConvWarps;
+    const int q4 = e & 3;
+    const int cs = e >> 2;                  // column slice
+    const int r = 32 * q4 + lane;           // row within the tile
     uint32_t gcount = 0;
+    uint32_t sc_use = 0;  // scale-ring entries consumed
+    uint8_t* const priv = smem + kPrivOff + e * kPrivBytes;
     bool ok = true;
-    int f_tile = blockIdx.x, f_g = 0;  // the fetch cursor walks the stream in order
-    auto fetch = [&]() -> float2 {
-      float2 v = make_float2(0.0f, 0.0f);
-      if (f_tile < num_tiles) {
-        if (et < kTileN)
-          v = __ldg(p.swp + static_cast<size_t>(f_g) * p.n_pad + (f_tile / num_m) * kTileN + et);
-        else
-          v.x = __half2float(p.sx[static_cast<size_t>(f_g) * p.m_pad + (f_tile % num_m) * kTileM + et - kTileN]);
-        if (++f_g == groups) {
-          f_g = 0;
-          f_tile += gridDim.x;
-        }
-      }
-      return v;
-    };
-    auto put = [&](int slot, float2 v) {
-      if (et < kTileN)
-        sc_sw[slot * kTileN + et] = v;
-      else
-        sc_sx[slot * kTileM + et - kTileN] = v.x;
-    };
-    static_assert(kScaleAhead == 4 && kScaleSlots == 8, "queue depth");
-    for (int t = 0; t < kScaleAhead; ++t) put(t, fetch());
-    float2 q0 = fetch(), q1 = fetch(), q2 = fetch(), q3 = fetch();
-    uint32_t ti = 0;  // stream index of the next group (wraps harmlessly: slots are ti % 8)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
       const int row = m0 + r;
-      float acc[64];
+      const int nc = n0 + 32 * cs;  // first column of this warp
+      float acc[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
+      for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
       const int uses = groups + (p.n_lora > 0 ? 1 : 0);
       for (int g = 0; g < uses; ++g, ++gcount) {
-        int sb = 0;
+        float sxr = 0.0f;
+        // (s_w, -magic s_w) of two columns per entry, broadcast reads of the
+        // warp's private copy
+        const float4* swq = reinterpret_cast<const float4*>(priv);
         if (g < groups) {
-          put((ti + kScaleAhead) % kScaleSlots, q0);  // past the stream's end: harmless zeros
-          named_bar_sync(1, 32 * kI4EpiWarps);       // publishes entry ti
-          q0 = q1;
-          q1 = q2;
-          q2 = q3;
-          q3 = fetch();
-          sb = static_cast<int>(ti % kScaleSlots);
-          ++ti;
+          // copy this warp's scales out of the ring entry, then release it:
+          // the stores consume the loaded values, so every load of the entry
+          // has completed before the arrival that lets the producer's next
+          // bulk copy overwrite it
+          const uint32_t ss = sc_use % kScaleSlots;
+          if (!mbar_wait(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) { ok = false; break; }
+          const uint8_t* sb = smem + kScaleOff + ss * kScaleSlotBytes;
+          reinterpret_cast<float2*>(priv)[lane] = reinterpret_cast<const float2*>(sb)[32 * cs + lane];
+          reinterpret_cast<float*>(priv + 256)[lane] =
+              __half2float(reinterpret_cast<const __half*>(sb + kTileN * 8)[r]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sc_empty[ss]);
+          ++sc_use;
+          sxr = reinterpret_cast<const float*>(priv + 256)[lane];
         }
         const uint32_t buf = gcount % kAccBufs;
         if (!mbar_wait(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const float sxr = sc_sx[sb * kTileM + r];
-        const float4* swq = reinterpret_cast<const float4*>(sc_sw + sb * kTileN + 64 * ch);  // broadcast
+        uint32_t P[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + buf * kTileN + 32 * cs, P);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the products are in registers: free the buffer
+        if (g < groups) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // 32 columns at a time
-          uint32_t P[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + buf * kTileN + 64 * ch + 32 * hh, P);
-          tmem_ld_wait();
-          if (hh == 1) {  // both halves read: the accumulator is free
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);
+          for (int c = 0; c < 32; c += 2) {
+            const float4 t = swq[c / 2];
+            // RN(P s_w) exactly: bits(magic) + P is the float magic + P
+            const float u0 = __fmaf_rn(__int_as_float(static_cast<int>(P[c]) + 0x4B400000), t.x, t.y);
+            const float u1 = __fmaf_rn(__int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000), t.z, t.w);
+            acc[c] = __fmaf_rn(u0, sxr, acc[c]);
+            acc[c + 1] = __fmaf_rn(u1, sxr, acc[c + 1]);
           }
-          if (g < groups) {
+          __syncwarp();  // the private copy is rewritten at the next group
+        } else {  // the lora-up, fp32
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float4 t = swq[(32 * hh + c) / 2];  // (s_w, -magic s_w) of two columns
-              // RN(P s_w) exactly: bits(magic) + P is the float magic + P
-              const float u0 = __fmaf_rn(__int_as_float(static_cast<int>(P[c]) + 0x4B400000), t.x, t.y);
-              const float u1 = __fmaf_rn(__int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000), t.z, t.w);
-              acc[32 * hh + c] = __fmaf_rn(u0, sxr, acc[32 * hh + c]);
-              acc[32 * hh + c + 1] = __fmaf_rn(u1, sxr, acc[32 * hh + c + 1]);
-            }
-          } else {  // the lora-up, fp32
-#pragma unroll
-            for (int c = 0; c < 32; ++c) acc[32 * hh + c] = __fadd_rn(acc[32 * hh + c], __uint_as_float(P[c]));
-          }
+          for (int c = 0; c < 32; ++c) acc[c] = __fadd_rn(acc[c], __uint_as_float(P[c]));
         }
       }
       if (!ok) break;
       if constexpr (kQkv) {
         // y = acc + b in place (N is a multiple of 128 here), then in Q / K
-        // tiles the head's RMS normalisation and rotary embedding; the two
-        // column halves of a row add their sums of squares through shared
-        // memory (the lower half first).  Every epilogue warp works on the
-        // same tile, so the barriers are uniform; the slot is next written
-        // after the next tile's first scale barrier.
-        const int nc = n0 + 64 * ch;
+        // tiles the head's RMS normalisation and rotary embedding.  A row's
+        // head is the whole tile: the four column slices of a lane quarter
+        // add their sums of squares through shared memory in slice order.
+        // Every epilogue warp works on the same tile, so the barriers are
+        // uniform; the slot is next written after this tile's second
+        // barrier, which every reader has passed.
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = __fadd_rn(acc[c], __ldg(p.bias + nc + c));
+        for (int c = 0; c < 32; ++c) acc[c] = __fadd_rn(acc[c], __ldg(p.bias + nc + c));
         if (n0 < p.qk_cols) {
           float ss = 0.0f;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) ss = __fmaf_rn(acc[c], acc[c], ss);
-          float* slot = red_s + q4 * 32 + lane;
-          if (ch) *slot = ss;
+          for (int c = 0; c < 32; ++c) ss = __fmaf_rn(acc[c], acc[c], ss);
+          red_s[(q4 * 4 + cs) * 32 + lane] = ss;
           named_bar_sync(2, 32 * kI4EpiWarps);
-          if (!ch) *slot = __fadd_rn(ss, *slot);
+          const float tot = __fadd_rn(__fadd_rn(red_s[(q4 * 4 + 0) * 32 + lane], red_s[(q4 * 4 + 1) * 32 + lane]),
+                                      __fadd_rn(red_s[(q4 * 4 + 2) * 32 + lane], red_s[(q4 * 4 + 3) * 32 + lane]));
           named_bar_sync(2, 32 * kI4EpiWarps);
-          const float rs = rsqrtf(__fmaf_rn(*slot, 1.0f / 128.0f, p.eps));
-          const float4* wn = reinterpret_cast<const float4*>((n0 < p.qk_cols / 2 ? p.norm_q : p.norm_k) + 64 * ch);
+          const float rs = rsqrtf(__fmaf_rn(tot, 1.0f / 128.0f, p.eps));
+          const float4* wn = reinterpret_cast<const float4*>((n0 < p.qk_cols / 2 ? p.norm_q : p.norm_k) + 32 * cs);
           // frequency-major rotary tables: one line per frequency per warp
           const bool in_rows = row < p.M;
-          const size_t trow = static_cast<size_t>(32 * ch) * p.M + (in_rows ? row : 0);
+          const size_t trow = static_cast<size_t>(16 * cs) * p.M + (in_rows ? row : 0);
           const float* ct = p.rope_cos + trow;
           const float* st = p.rope_sin + trow;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {  // four pairs per step
+          for (int q = 0; q < 4; ++q) {  // four pairs per step
             float cc[4], sc[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -400,13 +419,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       }
       if (row < p.M) {
 #pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          const int n = n0 + 64 * ch + c;
+        for (int c = 0; c < 32; c += 8) {
+          const int n = nc + c;
           if (n >= p.N) break;
           float y[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            y[e] = kQkv ? acc[c + e] : __fadd_rn(acc[c + e], n + e < p.N ? __ldg(p.bias + n + e) : 0.0f);
+          for (int j = 0; j < 8; ++j)
+            y[j] = kQkv ? acc[c + j] : __fadd_rn(acc[c + j], n + j < p.N ? __ldg(p.bias + n + j) : 0.0f);
           if (n + 8 <= p.N && (p.N & 7) == 0) {
             if constexpr (kF32Out) {
               float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + static_cast<size_t>(row) * p.N + n);
@@ -422,11 +441,11 @@ __global__ void __launch_bounds__(kI4Threads, 1)
               *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + static_cast<size_t>(row) * p.N + n) = o;
             }
           } else {
-            for (int e = 0; e < 8 && n + e < p.N; ++e) {
+            for (int j = 0; j < 8 && n + j < p.N; ++j) {
               if constexpr (kF32Out)
-                static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n + e] = y[e];
+                static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n + j] = y[j];
               else
-                static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n + e] = __float2bfloat16_rn(y[e]);
+                static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n + j] = __float2bfloat16_rn(y[j]);
             }
           }
         }
@@ -439,6 +458,8 @@ teardown:
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kI4Stages; ++s)
       if (issued_mask & (1u << s)) mbar_wait_limited(&full[s], (issued_par >> s) & 1u, 200000000ull);
+    for (int s = 0; s < kScaleSlots; ++s)
+      if (sc_mask & (1u << s)) mbar_wait_limited(&sc_full[s], (sc_par >> s) & 1u, 200000000ull);
   }
   if (warp == 1) {
     if (elect_one()) {
