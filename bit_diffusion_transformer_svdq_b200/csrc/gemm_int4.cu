@@ -352,14 +352,18 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the products are in registers: free the buffer
         if (g < groups) {
+          const float2 sx2 = make_float2(sxr, sxr);
 #pragma unroll
           for (int c = 0; c < 32; c += 2) {
             const float4 t = swq[c / 2];
-            // RN(P s_w) exactly: bits(magic) + P is the float magic + P
-            const float u0 = __fmaf_rn(__int_as_float(static_cast<int>(P[c]) + 0x4B400000), t.x, t.y);
-            const float u1 = __fmaf_rn(__int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000), t.z, t.w);
-            acc[c] = __fmaf_rn(u0, sxr, acc[c]);
-            acc[c + 1] = __fmaf_rn(u1, sxr, acc[c + 1]);
+            // RN(P s_w) exactly: bits(magic) + P is the float magic + P; two
+            // columns per packed FMA
+            const float2 f = make_float2(__int_as_float(static_cast<int>(P[c]) + 0x4B400000),
+                                         __int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000));
+            const float2 u = __ffma2_rn(f, make_float2(t.x, t.z), make_float2(t.y, t.w));
+            const float2 a = __ffma2_rn(u, sx2, make_float2(acc[c], acc[c + 1]));
+            acc[c] = a.x;
+            acc[c + 1] = a.y;
           }
           __syncwarp();  // the private copy is rewritten at the next group
         } else {  // the lora-up, fp32
