@@ -22,10 +22,13 @@ import numpy as np
 EXACT_MAX_DIM = 1024
 
 
-def truncated_svd(A: np.ndarray, r: int, power_steps: int = 4, oversample: int = 16, seed: int = 1234):
+def truncated_svd(A: np.ndarray, r: int, power_steps: int = 4, oversample: int = 16, seed: int = 1234,
+                  omega: np.ndarray | None = None, iterate: bool = False):
     """Return (U_r, s_r, V_r) of the fp64 matrix A (m x n): A ~ U_r diag(s_r) V_r^T.
 
-    U_r is m x r, V_r is n x r, s_r is non-increasing.
+    U_r is m x r, V_r is n x r, s_r is non-increasing.  `omega` (n x ell)
+    replaces the seeded Gaussian start block of the subspace iteration, and
+    `iterate` selects that iteration also for small matrices.
     """
     A = np.asarray(A, dtype=np.float64)
     m, n = A.shape
@@ -34,12 +37,14 @@ def truncated_svd(A: np.ndarray, r: int, power_steps: int = 4, oversample: int =
         return np.zeros((m, 0)), np.zeros(0), np.zeros((n, 0))
     if r > min(m, n):
         raise ValueError("rank larger than the matrix")
-    if min(m, n) <= EXACT_MAX_DIM:
+    if min(m, n) <= EXACT_MAX_DIM and not iterate and omega is None:
         U, s, Vt = np.linalg.svd(A, full_matrices=False)
         return U[:, :r], s[:r], Vt[:r].T
-    rng = np.random.Generator(np.random.PCG64(seed))
-    ell = min(r + oversample, min(m, n))
-    Q, _ = np.linalg.qr(A @ rng.standard_normal((n, ell)))
+    if omega is None:
+        rng = np.random.Generator(np.random.PCG64(seed))
+        ell = min(r + oversample, min(m, n))
+        omega = rng.standard_normal((n, ell))
+    Q, _ = np.linalg.qr(A @ np.asarray(omega, dtype=np.float64))
     for _ in range(power_steps):
         Z, _ = np.linalg.qr(A.T @ Q)
         Q, _ = np.linalg.qr(A @ Z)

@@ -67,10 +67,12 @@ def smooth_activation(x: np.ndarray, inv_lam: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float32) * np.asarray(inv_lam, dtype=np.float32)[None, :]
 
 
-def lowrank_factors(w: np.ndarray, lam: np.ndarray, rank: int):
-    """(L1 stored r x K, L2 stored N x r), both bf16 values held in fp32."""
+def lowrank_factors(w: np.ndarray, lam: np.ndarray, rank: int, omega: np.ndarray | None = None,
+                    power_steps: int = 4):
+    """(L1 stored r x K, L2 stored N x r), both bf16 values held in fp32.
+    With `omega` (N x ell) the subspace iteration starts from that block."""
     wt = smooth_weight(w, lam).astype(np.float64)  # N x K
-    U, s, V = truncated_svd(wt.T, rank)  # wt^T = U S V^T, U: K x r, V: N x r
+    U, s, V = truncated_svd(wt.T, rank, power_steps=power_steps, omega=omega)  # wt^T = U S V^T
     L1 = F.bf16_rn((U * s[None, :]).T).astype(np.float32)  # r x K
     L2 = F.bf16_rn(V).astype(np.float32)  # N x r
     return L1, L2

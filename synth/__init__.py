@@ -29,6 +29,7 @@ __all__ = [
     "bf16_bits_from_f32",
     "f32_from_bf16_bits",
     "qkv_prologue_inputs",
+    "svd_start_block",
 ]
 
 
@@ -183,3 +184,11 @@ def awq_alpha(K: int, seed: int) -> np.ndarray:
     near 1), drawn from (seed, K)."""
     rng = np.random.default_rng([seed, K, 11])
     return np.exp(rng.uniform(-0.5, 0.5, K)).astype(np.float32)
+
+
+def svd_start_block(n: int, ell: int, seed: int) -> np.ndarray:
+    """The Gaussian start block of the randomized subspace iteration that
+    factorises the smoothed weight (n x ell fp32, n = output features),
+    drawn from (seed, n, ell)."""
+    rng = np.random.default_rng([seed, n, ell, 13])
+    return rng.standard_normal((n, ell)).astype(np.float32)

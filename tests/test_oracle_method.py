@@ -168,3 +168,23 @@ def test_error_falls_as_rank_grows(precision):
     # with a rank-4 spike in W the branch must take most of the error away;
     # with a purely Gaussian W it can only shave the top of the spectrum
     assert errs[-1] < (0.5 if precision == "nvfp4" else 0.95) * errs[0], errs
+
+
+def test_subspace_iteration_matches_exact_svd_on_a_gapped_spectrum():
+    """The subspace path (forced on a small matrix, with a given start
+    block) recovers the top singular triplets of a matrix with a clear gap
+    after r: singular values to 1e-10 and the rank-r product to 1e-9."""
+    rng = np.random.default_rng(4)
+    m, n, r = 300, 200, 8
+    U0, _ = np.linalg.qr(rng.standard_normal((m, m)))
+    V0, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    s0 = np.concatenate([np.linspace(50, 20, r), 0.5 * np.exp(-np.arange(n - r) / 40.0)])
+    A = (U0[:, :n] * s0[None, :]) @ V0.T
+    omega = rng.standard_normal((n, r + 8))
+    U, s, V = S.truncated_svd(A, r, omega=omega)
+    assert np.allclose(s, s0[:r], rtol=1e-10)
+    Ue, se, Vte = np.linalg.svd(A, full_matrices=False)
+    assert np.allclose((U * s) @ V.T, (Ue[:, :r] * se[:r]) @ Vte[:r], rtol=0, atol=1e-9 * s0[0])
+    # the same start block through the seeded path gives the same result
+    U2, s2, V2 = S.truncated_svd(A, r, oversample=8, seed=9, iterate=True)
+    assert np.allclose(s2, s0[:r], rtol=1e-10)
