@@ -170,18 +170,19 @@ def run_ours(args, li, rank, world, local_rank):
     lam = torch.empty(K, dtype=torch.float32, device=dev)
     scratch = torch.empty(2 * K, dtype=torch.float32, device=dev)
     svdq.svdq_smoothing_lambda(X, W, lam, scratch)
-    # Stand-in for the offline factoriser: rank-r factors of W_til^T from
-    # torch's randomized SVD (fp32), rounded to bf16.
-    torch.manual_seed(0)
-    Wt = (W * lam[None, :]).t().contiguous()
-    U, S, Vv = torch.svd_lowrank(Wt, q=r + 16, niter=4)
-    L1 = (U[:, :r] * S[None, :r]).t().contiguous().to(torch.bfloat16).view(torch.int16)
-    L2 = Vv[:, :r].contiguous().to(torch.bfloat16).view(torch.int16)
+    # the offline factoriser: rank-r factors of W_til^T by the library's
+    # GPU subspace iteration from a seeded start block
+    L1 = torch.empty((r, K), dtype=torch.int16, device=dev)
+    L2 = torch.empty((N, r), dtype=torch.int16, device=dev)
+    omega = torch.from_numpy(synth.svd_start_block(N, r + 16, SEED)).to(dev)
+    lr_ws = svdq.alloc_workspace(None, 0, dev, nbytes=svdq.svdq_lowrank_workspace_bytes(N, K))
+    svdq.svdq_lowrank_factors(W, lam, r, omega, L1, L2, lr_ws)
+    del lr_ws, omega
     w = svdq.prepare_layer(W, lam, L1, L2, bias, r)
     gx_t = torch.empty(1, dtype=torch.float32, device=dev)
     svdq.svdq_act_global_scale(w, X, gx_t)
     gx = float(gx_t.item())
-    del W, Wt, U, S, Vv
+    del W
 
     ws = svdq.alloc_workspace(w, M, dev)
     qx = ws
@@ -331,6 +332,8 @@ def run_stack(args, rank, world, local_rank):
     stream = torch.cuda.current_stream()
     M = synth.WORKLOADS["stack_qkv"].M
     layers = []
+    lr_ws = svdq.alloc_workspace(None, 0, dev, nbytes=max(
+        svdq.svdq_lowrank_workspace_bytes(synth.WORKLOADS[n].N, synth.WORKLOADS[n].K) for n in synth.STACK_LAYERS))
     for blk in range(args.blocks):
         for j, name in enumerate(synth.STACK_LAYERS):
             shp = synth.WORKLOADS[name]
@@ -345,14 +348,15 @@ def run_stack(args, rank, world, local_rank):
             lam = torch.empty(K, dtype=torch.float32, device=dev)
             scratch = torch.empty(2 * K, dtype=torch.float32, device=dev)
             svdq.svdq_smoothing_lambda(X, W, lam, scratch)
-            U, S, Vv = torch.svd_lowrank((W * lam[None, :]).t(), q=r + 16, niter=4)
-            L1 = (U[:, :r] * S[None, :r]).t().contiguous().to(torch.bfloat16).view(torch.int16)
-            L2 = Vv[:, :r].contiguous().to(torch.bfloat16).view(torch.int16)
+            L1 = torch.empty((r, K), dtype=torch.int16, device=dev)
+            L2 = torch.empty((N, r), dtype=torch.int16, device=dev)
+            omega = torch.randn(N, r + 16, generator=g, device=dev)
+            svdq.svdq_lowrank_factors(W, lam, r, omega, L1, L2, lr_ws)
             w = svdq.prepare_layer(W, lam, L1, L2, b, r)
             gx_t = torch.empty(1, dtype=torch.float32, device=dev)
             svdq.svdq_act_global_scale(w, X, gx_t)
             layers.append((w, X, float(gx_t.item()), N, K))
-            del W, Xf, U, S, Vv
+            del W, Xf, omega
     torch.cuda.empty_cache()
     ws_bytes = max(svdq.svdq_workspace_bytes(w, M) for (w, _, _, _, _) in layers[:4])
     ws = svdq.alloc_workspace(layers[0][0], M, dev, nbytes=ws_bytes)

@@ -184,6 +184,30 @@ svdq_status svdq_smoothing_lambda(const uint16_t* X, int32_t M, const float* W, 
   return from_cuda(launch_smoothing_lambda(X, M, W, N, K, lambda, scratch, static_cast<cudaStream_t>(stream)));
 }
 
+size_t svdq_lowrank_workspace_bytes(int32_t N, int32_t K) {
+  if (N <= 0 || K <= 0) return 0;
+  return lowrank_workspace_bytes(N, K);
+}
+
+svdq_status svdq_lowrank_factors(const float* W, int32_t N, int32_t K, const float* lambda, int32_t rank,
+                                 int32_t oversample, int32_t power_steps, const float* omega, uint16_t* L1,
+                                 uint16_t* L2, void* workspace, size_t ws_bytes, void* stream) {
+  if (!W || !lambda || !omega || !L1 || !L2 || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || rank < 1 || rank % 8 != 0 || oversample < 0 || power_steps < 0 || power_steps > 16)
+    return SVDQ_ERR_SHAPE;
+  const int ell = rank + oversample;
+  if (ell > 64 || ell > N || ell > K) return SVDQ_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(lambda) || !aligned16(omega) || !aligned16(L1) || !aligned16(L2) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return SVDQ_ERR_ALIGNMENT;
+  if (ws_bytes < lowrank_workspace_bytes(N, K)) return SVDQ_ERR_WORKSPACE;
+  int dev;
+  svdq_status st = current_device(&dev);
+  if (st != SVDQ_OK) return st;
+  return from_cuda(launch_lowrank(W, N, K, lambda, rank, ell, power_steps, omega, L1, L2, workspace,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, const float* lambda, const uint16_t* L1,
                                  const uint16_t* L2, const uint16_t* bias, void* storage, size_t storage_bytes,
                                  svdq_weights** out, void* stream) {

@@ -80,6 +80,9 @@ cudaError_t launch_quantize(const svdq_weights* w, const uint16_t* X, int M, flo
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
                               const float* lora_act, int M, void* Y, int out_dtype, const svdq_qkv_prologue* pro,
                               cudaStream_t s);
+size_t lowrank_workspace_bytes(int N, int K);
+cudaError_t launch_lowrank(const float* W, int N, int K, const float* lambda, int rank, int ell, int power_steps,
+                           const float* omega, uint16_t* L1, uint16_t* L2, void* workspace, cudaStream_t s);
 cudaError_t launch_awq_gemv(const svdq_weights* w, const uint16_t* X, int M, void* Y, int out_dtype, cudaStream_t s);
 cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* lora_act, int M,
                              void* Y, int out_dtype, const svdq_qkv_prologue* pro, cudaStream_t s);

@@ -92,6 +92,8 @@ _SIGS = {
     "svdq_linear_forward_qkv": (_I, [_P, _P, _I, _F, ctypes.POINTER(QkvPrologue), _P, _I, _P, _Z, _P]),
     "svdq_linear_forward_noalloc": (_I, [_P, _P, _I, _F, _P, _I, _P]),
     "svdq_awq_w4a16_forward": (_I, [_P, _P, _I, _P, _I, _P]),
+    "svdq_lowrank_workspace_bytes": (_Z, [_I, _I]),
+    "svdq_lowrank_factors": (_I, [_P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, _Z, _P]),
     "svdq_device_status": (_I, [_P, _P]),
     "svdq_selftest_bounded_wait": (_I, [_P]),
 }
@@ -254,6 +256,22 @@ def svdq_awq_w4a16_forward(w: Weights, X, M: int, Y, out_dtype: int = SVDQ_OUT_B
            "svdq_awq_w4a16_forward")
 
 
+def svdq_lowrank_workspace_bytes(N: int, K: int) -> int:
+    return load_library().svdq_lowrank_workspace_bytes(N, K)
+
+
+def svdq_lowrank_factors(W, lam, rank: int, omega, L1, L2, workspace, oversample: int = 16, power_steps: int = 4,
+                         stream=None) -> None:
+    """Rank-`rank` factors of the smoothed weight (W: N x K fp32, lam: K,
+    omega: N x (rank + oversample) fp32 start block) into L1 (rank x K bf16
+    bits) and L2 (N x rank bf16 bits)."""
+    N, K = W.shape
+    _check(load_library().svdq_lowrank_factors(_ptr(W), N, K, _ptr(lam), rank, oversample, power_steps, _ptr(omega),
+                                               _ptr(L1), _ptr(L2), _ptr(workspace),
+                                               workspace.numel() * workspace.element_size(), _stream(stream)),
+           "svdq_lowrank_factors")
+
+
 def svdq_device_status(w: Weights, stream=None) -> int:
     return load_library().svdq_device_status(w.handle, _stream(stream))
 
@@ -282,9 +300,10 @@ def prepare_layer(W: torch.Tensor, lam: torch.Tensor, L1: torch.Tensor | None, L
     return svdq_prepare_weights(desc, W, lam, L1, L2, bias, storage, stream)
 
 
-def alloc_workspace(w: Weights, M: int, device, nbytes: int | None = None) -> torch.Tensor:
+def alloc_workspace(w: Weights | None, M: int, device, nbytes: int | None = None) -> torch.Tensor:
     """A 1024-aligned device workspace of svdq_workspace_bytes(w, M) bytes
-    (or `nbytes`, e.g. the largest over several layers sharing it)."""
+    (or `nbytes`, e.g. the largest over several layers sharing it, or the
+    factoriser's svdq_lowrank_workspace_bytes)."""
     n = svdq_workspace_bytes(w, M) if nbytes is None else nbytes
     buf = torch.empty(n + 1024, dtype=torch.uint8, device=device)
     off = (-buf.data_ptr()) % 1024

@@ -163,6 +163,28 @@ SVDQ_API svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const flo
                                  const uint16_t* L1, const uint16_t* L2, const uint16_t* bias,
                                  void* storage, size_t storage_bytes, svdq_weights** out, void* stream);
 
+/* The low-rank factors L1 (rank x K) and L2 (N x rank) that
+ * svdq_prepare_weights takes, computed on the GPU: a truncated SVD of the
+ * smoothed weight W_til^T = (RN32(W * lambda))^T (K x N) by randomized block
+ * subspace iteration (Halko, Martinsson and Tropp 2011; the pages name the
+ * method, "Nunchaku und SVDQuant", but not the factorisation):
+ *     Q = orth(W_til^T Omega);  power_steps times: Z = orth(W_til Q),
+ *     Q = orth(W_til^T Z);  B = Q^T W_til^T = U_b diag(s) V^T;
+ *     L1 = bf16((Q U_b)_r diag(s_r))^T,  L2 = bf16(V_r)
+ * with orth() two passes of Cholesky QR (fp64 Gram matrices) and the small
+ * SVD from the fp64 eigendecomposition of B B^T.  The signs of matching
+ * columns of U and V are arbitrary; L2 L1 is not.
+ * Inputs [device]: W N x K fp32, lambda K fp32, omega N x ell fp32 (the
+ * start block, e.g. standard normal draws; ell = rank + oversample).
+ * Outputs [device]: L1 rank x K bf16, L2 N x rank bf16.  workspace [device]
+ * >= svdq_lowrank_workspace_bytes(N, K) bytes, 256-byte aligned.
+ * Limits: 1 <= rank, rank % 8 == 0, oversample >= 0, ell <= 64,
+ * ell <= min(N, K), 0 <= power_steps <= 16.  Asynchronous on `stream`. */
+SVDQ_API size_t svdq_lowrank_workspace_bytes(int32_t N, int32_t K);
+SVDQ_API svdq_status svdq_lowrank_factors(const float* W, int32_t N, int32_t K, const float* lambda, int32_t rank,
+                                 int32_t oversample, int32_t power_steps, const float* omega, uint16_t* L1,
+                                 uint16_t* L2, void* workspace, size_t ws_bytes, void* stream);
+
 /* Frees the host handle (not the caller's device storage).  NULL is a no-op. */
 SVDQ_API void svdq_weights_destroy(svdq_weights* w);
 
