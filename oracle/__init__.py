@@ -32,5 +32,7 @@ Modules:
   qkv      - the attention prologue of the fused QKV projection (per-head
              RMS normalisation of Q and K, rotary embedding)
   awq      - the awq_w4a16 layer (INT4 group-64 weights, 16-bit activations)
+  chain    - the dynamic activation tensor scale and chained layers (an
+             activation between them, the next layer's amax)
 """
-from . import awq, formats, qkv, quant, svd, svdq  # noqa: F401
+from . import awq, chain, formats, qkv, quant, svd, svdq  # noqa: F401
