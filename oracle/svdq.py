@@ -144,9 +144,12 @@ class ActQuant:
 
 
 def quantize_activations(x, prep: Prepared, g_x=None) -> ActQuant:
-    """Smoothing + 4-bit quantisation of X_hat + lora-down X L1s^T."""
+    """Smoothing + 4-bit quantisation of X_hat + lora-down X L1s^T.  NVFP4
+    with g_x None: the dynamic tensor scale of this very X."""
     xh = smooth_activation(x, prep.inv_lam)
     if prep.precision == "nvfp4":
+        if g_x is None:
+            g_x = act_global_scale(x, prep.inv_lam)
         qx, sx = Q.nvfp4_quantize(xh, np.float32(g_x))
     else:
         qx, sx = Q.int4_quantize(xh)
@@ -168,7 +171,10 @@ def gemm_unscaled(a: ActQuant, prep: Prepared) -> np.ndarray:
 
 
 def forward_from_codes(a: ActQuant, prep: Prepared, g_x=None) -> np.ndarray:
-    """Y* = g_x g_w (4-bit product) + (X L1s^T) L2^T + b, in fp64."""
+    """Y* = g_x g_w (4-bit product) + (X L1s^T) L2^T + b, in fp64.  NVFP4
+    needs the tensor scale the codes were made with."""
+    if prep.precision == "nvfp4" and g_x is None:
+        raise ValueError("NVFP4 codes need their tensor scale g_x")
     S = gemm_unscaled(a, prep)
     if prep.precision == "nvfp4":
         S = S * (float(np.float32(g_x)) * float(prep.g_w))
@@ -177,6 +183,10 @@ def forward_from_codes(a: ActQuant, prep: Prepared, g_x=None) -> np.ndarray:
 
 
 def forward(x, prep: Prepared, g_x=None) -> np.ndarray:
+    """The layer in fp64; NVFP4 with g_x None takes the dynamic tensor
+    scale of this X."""
+    if g_x is None and prep.precision == "nvfp4":
+        g_x = act_global_scale(x, prep.inv_lam)
     return forward_from_codes(quantize_activations(x, prep, g_x), prep, g_x)
 
 

@@ -97,3 +97,17 @@ def test_chain_scale_matches_calibration_formula():
     # GELU output is bounded below by its minimum, about -0.17
     assert ya.min() > -0.2
     assert yb.shape == (40, 64) and np.all(np.isfinite(yb))
+
+
+def test_dynamic_scale_is_the_default():
+    li = synth.make_layer("mlp_up", 8, M=33, K=128, N=64)
+    lam = V.smoothing_lambda(li.x, li.w)
+    p = V.prepare_weights(li.w, lam, *V.lowrank_factors(li.w, lam, 8), li.bias)
+    g = V.act_global_scale(li.x, p.inv_lam)
+    a0, a1 = V.quantize_activations(li.x, p, None), V.quantize_activations(li.x, p, g)
+    assert np.array_equal(a0.qx, a1.qx) and np.array_equal(a0.sx, a1.sx)
+    assert np.any(a0.qx != 0)
+    assert np.array_equal(V.forward(li.x, p), V.forward(li.x, p, g))
+    # a different scale gives different scale codes
+    a2 = V.quantize_activations(li.x, p, np.float32(g * 2))
+    assert not np.array_equal(a2.sx, a1.sx)
