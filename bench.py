@@ -321,7 +321,14 @@ def run_stack(args, rank, world, local_rank):
     svdq_linear_forward, each with its own seeded weights, input and
     calibration (inputs are not chained: attention and norms are not part of
     the layer).  Weights and inputs are drawn on the GPU; preparation is
-    untimed.  One L2 read-flush before each timed step."""
+    untimed.  One L2 read-flush before each timed step.
+
+    --scale static: each layer's calibrated tensor scale (svdq_linear_forward).
+    --scale dynamic: every layer takes its scale from its own input on the
+    device (svdq_linear_forward_dyn: an amax pass, the quantiser, the GEMM).
+    --scale chain: dynamic, and the feed-forward is chained: the MLP up
+    epilogue applies the GELU and max-reduces the down layer's amax, and the
+    down layer quantises that output with it (no amax pass there)."""
     import torch
     import synth
     from bit_diffusion_transformer_svdq_b200 import svdq
@@ -363,9 +370,28 @@ def run_stack(args, rank, world, local_rank):
     Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (_, _, _, N, _) in layers[:4]}
     flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
 
+    words = torch.zeros(2, dtype=torch.float32, device=dev)
+    epis = {}
+    for i, (w, _, _, _, _) in enumerate(layers):
+        if i % 4 == 2:  # MLP up: GELU, and the amax of the down layer that follows
+            il = layers[i + 1][0].view().inv_lambda
+            epis[i] = svdq.make_epilogue_next(svdq.SVDQ_ACT_GELU_TANH, il, words[1:])
+
     def step():
-        for (w, X, gx, N, _) in layers:
-            svdq.svdq_linear_forward(w, X, M, gx, Ys[N], ws, ws.numel(), svdq.SVDQ_OUT_BF16, stream)
+        if args.scale == "static":
+            for (w, X, gx, N, _) in layers:
+                svdq.svdq_linear_forward(w, X, M, gx, Ys[N], ws, ws.numel(), svdq.SVDQ_OUT_BF16, stream)
+        elif args.scale == "dynamic":
+            for (w, X, _, N, _) in layers:
+                svdq.svdq_linear_forward_dyn(w, X, M, None, Ys[N], ws, ws.numel(), stream=stream)
+        else:
+            for i, (w, X, _, N, _) in enumerate(layers):
+                if i % 4 == 3:  # MLP down on the up layer's output and amax
+                    svdq.svdq_linear_forward_dyn(w, Ys[12288].view(torch.int16), M, words[1:], Ys[N], ws,
+                                                 ws.numel(), stream=stream)
+                else:
+                    svdq.svdq_linear_forward_dyn(w, X, M, None, Ys[N], ws, ws.numel(), epi=epis.get(i),
+                                                 stream=stream)
 
     for _ in range(args.warmup):
         flush.sum()
@@ -393,6 +419,10 @@ def run_stack(args, rank, world, local_rank):
     assert all(svdq.svdq_device_status(w) == 0 for (w, _, _, _, _) in layers)
     t_ms = _allreduce_max(sum(a.elapsed_time(b) for a, b in ts) / len(ts), world, dev)
     flops = sum(2.0 * M * N * K for (_, _, _, N, K) in layers)
+    # kernels per linear: quantiser + GEMM, plus the amax pass when the
+    # scale is dynamic (not for the chained down layers)
+    per_step = {"static": 2 * len(layers), "dynamic": 3 * len(layers),
+                "chain": 3 * len(layers) - len(layers) // 4}[args.scale]
     if rank == 0:
         print(json.dumps({
             "metric": "fused SVDQuant W4A4 linear effective TOPS, one denoising step of the block stack",
@@ -400,9 +430,10 @@ def run_stack(args, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
             "config": {"workload": f"{args.blocks} blocks x 4 linears (QKV, out, MLP up, down), M={M}, rank 32, nvfp4",
-                       "linears": len(layers), "l2": "flushed (256 MiB read) once before each step",
+                       "linears": len(layers), "tensor_scale": args.scale,
+                       "l2": "flushed (256 MiB read) once before each step",
                        "parallelism": f"replicas x{world}"},
-            "gpu_launches": 2 * len(layers) * args.steps, "clocks": clocks}), flush=True)
+            "gpu_launches": per_step * args.steps, "clocks": clocks}), flush=True)
 
 
 def run_awq(args, rank, world, local_rank):
@@ -499,6 +530,8 @@ def main():
                          "awq: the awq_w4a16 modulation projection")
     ap.add_argument("--batch", type=int, default=1, help="rows of the awq workload (images)")
     ap.add_argument("--blocks", type=int, default=57, help="blocks of the stack workload")
+    ap.add_argument("--scale", default="static", choices=["static", "dynamic", "chain"],
+                    help="activation tensor scale of the stack workload (see run_stack)")
     ap.add_argument("--qkv-prologue", action="store_true",
                     help="qkv workload: the GEMM also applies the QK-norm + rotary attention prologue")
     args = ap.parse_args()

@@ -313,45 +313,95 @@ svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t* X, int3
   return from_cuda(launch_act_global_scale(w, X, M, g_x, static_cast<cudaStream_t>(stream)));
 }
 
+svdq_status svdq_act_amax(const svdq_weights* w, const uint16_t* X, int32_t M, float* amax, void* stream) {
+  if (!w || !X || !amax || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
+  if (M <= 0) return SVDQ_ERR_SHAPE;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(amax) & 3u)) return SVDQ_ERR_ALIGNMENT;
+  int dev;
+  svdq_status st = current_device(&dev);
+  if (st != SVDQ_OK) return st;
+  return from_cuda(launch_act_amax(w, X, M, amax, static_cast<cudaStream_t>(stream)));
+}
+
 size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M) {
   if (!w || M < 0) return 0;
   const int64_t mp = m_pad_of(M);
   return w->desc.precision == SVDQ_NVFP4 ? nvfp4_scale_bytes(mp, w->desc.K) : int4_scale_bytes(mp, w->desc.K);
 }
 
-svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, uint8_t* qx,
-                                        void* sx, float* lora_act, void* stream) {
+namespace {
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Shared by the quantiser entry points.  `x_amax` (dynamic tensor scale)
+// replaces g_x for NVFP4; `zero_word` (may be null) is set to 0 by the
+// kernel before it ends.
+svdq_status quantize_entry(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, const float* x_amax,
+                           uint8_t* qx, void* sx, float* lora_act, float* zero_word, void* stream) {
   if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;  // 16-bit activations there
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
   if (!X || !qx || !sx || (w->rank_pad > 0 && !lora_act)) return SVDQ_ERR_INVALID_ARG;
-  if (w->desc.precision == SVDQ_NVFP4 && !(g_x > 0.0f && g_x < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
+  const bool nvfp4 = w->desc.precision == SVDQ_NVFP4;
+  if (nvfp4 && !x_amax && !(g_x > 0.0f && g_x < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(qx) || !aligned16(sx) || (lora_act && !aligned16(lora_act)))
     return SVDQ_ERR_ALIGNMENT;
+  if ((x_amax && !aligned4(x_amax)) || (zero_word && !aligned4(zero_word))) return SVDQ_ERR_ALIGNMENT;
   int dev;
   svdq_status st = current_device(&dev);
   if (st != SVDQ_OK) return st;
-  return from_cuda(launch_quantize(w, X, M, g_x, qx, sx, lora_act, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_quantize(w, X, M, x_amax ? 1.0f : g_x, nvfp4 ? x_amax : nullptr, qx, sx, lora_act,
+                                   zero_word, static_cast<cudaStream_t>(stream)));
+}
+
+// The epilogue extras' limits (see svdq.h).
+svdq_status check_epi(const svdq_weights* w, const svdq_epilogue_next* epi, const svdq_qkv_prologue* pro) {
+  if (!epi) return SVDQ_OK;
+  if (epi->activation != SVDQ_ACT_NONE && epi->activation != SVDQ_ACT_GELU_TANH) return SVDQ_ERR_INVALID_ARG;
+  if (!epi->next_inv_lambda != !epi->next_amax) return SVDQ_ERR_INVALID_ARG;
+  const bool asks = epi->activation != SVDQ_ACT_NONE || epi->next_amax;
+  if (asks && (pro || w->desc.precision != SVDQ_NVFP4)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned4(epi->next_inv_lambda) || !aligned4(epi->next_amax)) return SVDQ_ERR_ALIGNMENT;
+  return SVDQ_OK;
+}
+}  // namespace
+
+svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, uint8_t* qx,
+                                        void* sx, float* lora_act, void* stream) {
+  return quantize_entry(w, X, M, g_x, nullptr, qx, sx, lora_act, nullptr, stream);
+}
+
+svdq_status svdq_quantize_act_lora_down_dyn(const svdq_weights* w, const uint16_t* X, int32_t M, const float* x_amax,
+                                            uint8_t* qx, void* sx, float* lora_act, void* stream) {
+  if (w && w->desc.precision == SVDQ_NVFP4 && !x_amax) return SVDQ_ERR_INVALID_ARG;
+  return quantize_entry(w, X, M, 1.0f, x_amax, qx, sx, lora_act, nullptr, stream);
 }
 
 namespace {
 // Shared by the GEMM entry points: argument checks, then the launch.
-svdq_status gemm_entry(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x, const float* lora_act,
-                       int32_t M, const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* stream) {
+svdq_status gemm_entry(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x, const float* x_amax,
+                       const float* lora_act, int32_t M, const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi,
+                       void* Y, int32_t out_dtype, void* stream) {
   if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
+  const svdq_status ce = check_epi(w, epi, pro);
+  if (ce != SVDQ_OK) return ce;
   if (M == 0) return SVDQ_OK;
   if (!qx || !sx || !Y || (w->rank_pad > 0 && !lora_act)) return SVDQ_ERR_INVALID_ARG;
   if (out_dtype != SVDQ_OUT_BF16 && out_dtype != SVDQ_OUT_F32) return SVDQ_ERR_INVALID_ARG;
-  if (w->desc.precision == SVDQ_NVFP4 && !(g_x > 0.0f && g_x < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
+  const bool nvfp4 = w->desc.precision == SVDQ_NVFP4;
+  if (nvfp4 && !x_amax && !(g_x > 0.0f && g_x < 3.0e38f)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(qx) || !aligned16(sx) || !aligned16(Y) || (lora_act && !aligned16(lora_act)))
     return SVDQ_ERR_ALIGNMENT;
+  if (x_amax && !aligned4(x_amax)) return SVDQ_ERR_ALIGNMENT;
   int dev;
   svdq_status st = current_device(&dev);
   if (st != SVDQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (w->desc.precision == SVDQ_NVFP4)
-    return from_cuda(launch_gemm_nvfp4(w, qx, static_cast<const uint8_t*>(sx), g_x, lora_act, M, Y, out_dtype, pro, s));
+  if (nvfp4) {
+    const bool asks = epi && (epi->activation != SVDQ_ACT_NONE || epi->next_amax);
+    return from_cuda(launch_gemm_nvfp4(w, qx, static_cast<const uint8_t*>(sx), x_amax ? 1.0f : g_x, x_amax, lora_act,
+                                       M, Y, out_dtype, pro, asks ? epi : nullptr, s));
+  }
   return from_cuda(launch_gemm_int4(w, qx, sx, lora_act, M, Y, out_dtype, pro, s));
 }
 
@@ -370,7 +420,7 @@ svdq_status check_qkv(const svdq_weights* w, const svdq_qkv_prologue* pro) {
 
 svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
                                    const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream) {
-  return gemm_entry(w, qx, sx, g_x, lora_act, M, nullptr, Y, out_dtype, stream);
+  return gemm_entry(w, qx, sx, g_x, nullptr, lora_act, M, nullptr, nullptr, Y, out_dtype, stream);
 }
 
 svdq_status svdq_w4a4_gemm_lora_up_qkv(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
@@ -378,7 +428,18 @@ svdq_status svdq_w4a4_gemm_lora_up_qkv(const svdq_weights* w, const uint8_t* qx,
                                        int32_t out_dtype, void* stream) {
   const svdq_status st = check_qkv(w, pro);
   if (st != SVDQ_OK) return st;
-  return gemm_entry(w, qx, sx, g_x, lora_act, M, pro, Y, out_dtype, stream);
+  return gemm_entry(w, qx, sx, g_x, nullptr, lora_act, M, pro, nullptr, Y, out_dtype, stream);
+}
+
+svdq_status svdq_w4a4_gemm_lora_up_dyn(const svdq_weights* w, const uint8_t* qx, const void* sx, const float* x_amax,
+                                       const float* lora_act, int32_t M, const svdq_qkv_prologue* pro,
+                                       const svdq_epilogue_next* epi, void* Y, int32_t out_dtype, void* stream) {
+  if (w && w->desc.precision == SVDQ_NVFP4 && !x_amax) return SVDQ_ERR_INVALID_ARG;
+  if (pro) {
+    const svdq_status st = check_qkv(w, pro);
+    if (st != SVDQ_OK) return st;
+  }
+  return gemm_entry(w, qx, sx, 1.0f, x_amax, lora_act, M, pro, epi, Y, out_dtype, stream);
 }
 
 size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M) {
@@ -386,32 +447,51 @@ size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M) {
   const size_t qx = static_cast<size_t>(round_up(static_cast<int64_t>(M) * (w->desc.K / 2), 1024));
   const size_t sx = static_cast<size_t>(round_up(static_cast<int64_t>(svdq_act_scale_bytes(w, M)), 1024));
   const size_t la = static_cast<size_t>(round_up(static_cast<int64_t>(M) * w->rank_pad * 4, 1024));
-  return qx + sx + la;
+  return qx + sx + la + 1024;  // + the dynamic tensor scale's amax word
 }
 
 namespace {
-svdq_status forward_entry(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
-                          const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace, size_t ws_bytes,
-                          void* stream) {
+// The layer forward: quantiser then GEMM on one stream.  dyn: the dynamic
+// tensor scale from `x_amax`, or, when that is null, from an amax pass
+// into the workspace's last 1024 bytes.
+svdq_status forward_entry(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, bool dyn,
+                          const float* x_amax, const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi, void* Y,
+                          int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream) {
   if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
+  svdq_status st = check_epi(w, epi, pro);
+  if (st != SVDQ_OK) return st;
   if (M == 0) return SVDQ_OK;
   if (!workspace) return SVDQ_ERR_INVALID_ARG;
-  if (ws_bytes < svdq_workspace_bytes(w, M)) return SVDQ_ERR_WORKSPACE;
+  const size_t need = svdq_workspace_bytes(w, M);
+  if (ws_bytes < need) return SVDQ_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return SVDQ_ERR_ALIGNMENT;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* qx = ws;
   uint8_t* sx = qx + round_up(static_cast<int64_t>(M) * (w->desc.K / 2), 1024);
   float* la = reinterpret_cast<float*>(sx + round_up(static_cast<int64_t>(svdq_act_scale_bytes(w, M)), 1024));
-  svdq_status st = svdq_quantize_act_lora_down(w, X, M, g_x, qx, sx, w->rank_pad ? la : nullptr, stream);
+  float* amax_slot = reinterpret_cast<float*>(ws + need - 1024);
+  const bool nvfp4 = w->desc.precision == SVDQ_NVFP4;
+  float* next_amax = epi ? epi->next_amax : nullptr;
+  if (dyn && nvfp4 && !x_amax) {
+    if (!X) return SVDQ_ERR_INVALID_ARG;
+    if ((st = svdq_act_amax(w, X, M, amax_slot, stream)) != SVDQ_OK) return st;
+    x_amax = amax_slot;
+  }
+  if (next_amax && next_amax == x_amax) return SVDQ_ERR_INVALID_ARG;
+  // the quantiser zeroes the next layer's amax word (stream order puts the
+  // GEMM's max-reduction after it): no separate memset
+  st = quantize_entry(w, X, M, g_x, dyn && nvfp4 ? x_amax : nullptr, qx, sx, w->rank_pad ? la : nullptr, next_amax,
+                      stream);
   if (st != SVDQ_OK) return st;
-  return gemm_entry(w, qx, sx, g_x, w->rank_pad ? la : nullptr, M, pro, Y, out_dtype, stream);
+  return gemm_entry(w, qx, sx, g_x, dyn && nvfp4 ? x_amax : nullptr, w->rank_pad ? la : nullptr, M, pro, epi, Y,
+                    out_dtype, stream);
 }
 }  // namespace
 
 svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x, void* Y,
                                 int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream) {
-  return forward_entry(w, X, M, g_x, nullptr, Y, out_dtype, workspace, ws_bytes, stream);
+  return forward_entry(w, X, M, g_x, false, nullptr, nullptr, nullptr, Y, out_dtype, workspace, ws_bytes, stream);
 }
 
 svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
@@ -419,7 +499,17 @@ svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, in
                                     size_t ws_bytes, void* stream) {
   const svdq_status st = check_qkv(w, pro);
   if (st != SVDQ_OK) return st;
-  return forward_entry(w, X, M, g_x, pro, Y, out_dtype, workspace, ws_bytes, stream);
+  return forward_entry(w, X, M, g_x, false, nullptr, pro, nullptr, Y, out_dtype, workspace, ws_bytes, stream);
+}
+
+svdq_status svdq_linear_forward_dyn(const svdq_weights* w, const uint16_t* X, int32_t M, const float* x_amax,
+                                    const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi, void* Y,
+                                    int32_t out_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (pro) {
+    const svdq_status st = check_qkv(w, pro);
+    if (st != SVDQ_OK) return st;
+  }
+  return forward_entry(w, X, M, 1.0f, true, x_amax, pro, epi, Y, out_dtype, workspace, ws_bytes, stream);
 }
 
 svdq_status svdq_awq_w4a16_forward(const svdq_weights* w, const uint16_t* X, int32_t M, void* Y, int32_t out_dtype,

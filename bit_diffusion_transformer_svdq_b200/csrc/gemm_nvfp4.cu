@@ -36,6 +36,13 @@
 // (2i, 2i+1) by the row's rotary angle, all in fp32 before the one
 // rounding to the output type.
 //
+// Chained variant (a layer whose output feeds the next W4A4 layer, e.g. the
+// FLUX feed-forward's up-projection, GELU and down-projection): the
+// epilogue optionally applies the tanh-form GELU before the rounding and
+// reduces max |RN(y_stored * 1/lambda')| over its outputs (lambda' the next
+// layer's smoothing factors) into one device word, the next layer's
+// dynamic tensor-scale amax, with one atomic max per warp.
+//
 // TMEM columns (same in both CTAs): [0, 256) accumulator (this CTA's 128
 // rows), then one scale slot of 48 columns per ring stage: 16 columns of A
 // scales (this CTA's rows) and 32 of B scales (all 256 columns; each CTA
@@ -85,12 +92,36 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 
 constexpr uint32_t kIdescTf32 =
     (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 
+// epilogue variants
+constexpr int kModePlain = 0, kModeQkv = 1, kModeChain = 2, kModeChainGelu = 3;
+
+// GELU in its tanh form, 0.5 y (1 + tanh(u)) with u = sqrt(2/pi) (y +
+// 0.044715 y^3), through the identity 0.5 (1 + tanh(u)) = 1 / (1 + e^(-2u)):
+// y / (1 + 2^z), z = y (c0 + c1 y^2), c0 = -2 log2(e) sqrt(2/pi), c1 =
+// 0.044715 c0.  No cancellation for negative y (unlike 1 + tanh), so the
+// hardware exp2 and reciprocal keep the relative error near 1e-6.  z is
+// clamped so that 1 + 2^z stays finite.
+__device__ __forceinline__ float gelu_tanh(float y) {
+  const float z = fminf(__fmul_rn(y, __fmaf_rn(-0.10294324f, __fmul_rn(y, y), -2.3022082f)), 120.0f);
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(z));
+  return __fdividef(y, 1.0f + e);
+}
+
 struct GemmParams {
   const float* bias;
   void* Y;
   int* status;
   int M, N, K, n_lora;
   float gxgw;
+  // dynamic tensor scale: when set, gxgw = RN(RN(*x_amax / 2688) * g_w)
+  // (g_x = 1 for a zero amax)
+  const float* x_amax;
+  float g_w;
+  // chained variant: the next layer's 1/lambda (N values, or null) and the
+  // word its amax is max-reduced into
+  const float* next_il;
+  float* next_amax;
   int tma_store;  // Y rows are whole multiples of 16 bytes: store through tm_y
   // QKV attention prologue (the kQkv variant only)
   const float* norm_q;
@@ -101,12 +132,14 @@ struct GemmParams {
   int qk_cols;  // columns of Q and K (2 * heads * 128); K starts at qk_cols / 2
 };
 
-template <bool kF32Out, bool kQkv>
+template <bool kF32Out, int kMode, bool kDyn>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                       const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                       const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                       const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+  constexpr bool kQkv = kMode == kModeQkv;
+  constexpr bool kChain = kMode >= kModeChain;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + kBiasOff);
@@ -261,14 +294,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = (warp - 2) * 32 + lane;  // 0..511 over the epilogue warps
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* const stg = smem + kStagingOff + (warp - 2) * kStagingPerWarp;  // a 128-byte-swizzled box
+    // RN(g_x g_w): as given, or from the device amax (kept out of a register
+    // in the static variants, which sit at the register limit)
+    float gxgw = p.gxgw;
+    if constexpr (kDyn) {
+      const float a = *p.x_amax;
+      gxgw = __fmul_rn(a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f), p.g_w);
+    }
+    float amax_next = 0.0f;  // chained variant: max |y_stored / lambda'| over this thread's rows < M
     uint32_t acc_phase = 0;
     int tcount = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
       const int m0 = (tile % num_m) * BM + 128 * static_cast<int>(rank), n0 = (tile / num_m) * BN;
-      // the tile's 256 bias values, once, into this tile's half of the double buffer
-      float* bias_t = bias_s + (tcount & 1) * BN;
-      if (et < BN) bias_t[et] = n0 + et < p.N ? __ldg(p.bias + n0 + et) : 0.0f;
-      named_bar_sync(1, 32 * kEpiWarps);
+      float* bias_t;
+      if constexpr (!kChain) {
+        // the tile's 256 bias values, once, into this tile's half of the double buffer
+        bias_t = bias_s + (tcount & 1) * BN;
+        if (et < BN) bias_t[et] = n0 + et < p.N ? __ldg(p.bias + n0 + et) : 0.0f;
+        named_bar_sync(1, 32 * kEpiWarps);
+      } else {
+        // single buffers of the tile's bias and next-layer 1/lambda: written
+        // once every epilogue warp is past the previous tile (barrier 1),
+        // read after barrier 2
+        bias_t = bias_s;
+        float bz = 0.0f, lz = 0.0f;
+        if (et < BN && n0 + et < p.N) {
+          bz = __ldg(p.bias + n0 + et);
+          if (p.next_il != nullptr) lz = __ldg(p.next_il + n0 + et);
+        }
+        named_bar_sync(1, 32 * kEpiWarps);
+        if (et < BN) {
+          bias_s[et] = bz;
+          bias_s[BN + et] = lz;
+        }
+      }
       if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
       acc_phase ^= 1;
       tc_fence_after();
@@ -295,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // so every epilogue warp takes the same barriers)
 #pragma unroll
         for (int c = 0; c < kColsPerWarp; ++c)
-          v[c] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(v[c]), p.gxgw), bb[c]));
+          v[c] = __float_as_uint(__fadd_rn(__fmul_rn(__uint_as_float(v[c]), gxgw), bb[c]));
         if (n0 < p.qk_cols) {
           const int hcol = (part & 1) * kColsPerWarp;  // first column of this half within its head
           // rotary tables are frequency-major (pair i of token m at i * M + m):
@@ -350,10 +409,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // the dynamic variants also compute y in place first, so that the
+      // scale's register is free in the store loop
+      if constexpr (kMode == kModeChainGelu) {
+#pragma unroll
+        for (int c = 0; c < kColsPerWarp; ++c) {
+          const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[c]), gxgw), bb[c]);
+          v[c] = __float_as_uint(kMode == kModeChainGelu ? gelu_tanh(y) : y);
+        }
+      }
       // the value stored for column `col` of the warp's 64
       auto yv = [&](int col) -> float {
-        if constexpr (kQkv) return __uint_as_float(v[col]);
-        else return __fadd_rn(__fmul_rn(__uint_as_float(v[col]), p.gxgw), bb[col]);
+        if constexpr (kQkv || kMode == kModeChainGelu) return __uint_as_float(v[col]);
+        else return __fadd_rn(__fmul_rn(__uint_as_float(v[col]), gxgw), bb[col]);
+      };
+      // chained variant: max |y_stored / lambda'| over the rows < M (columns
+      // past N carry 1/lambda' = 0); the 1/lambda' buffer follows the bias
+      const bool row_ok = row < p.M;
+      auto track = [&](float ys, int col) {
+        if constexpr (kChain)
+          if (row_ok) amax_next = fmaxf(amax_next, fabsf(__fmul_rn(ys, bb[BN + col])));
       };
       if (p.tma_store) {
         // y rows into a 64-byte-wide swizzled box (32 rows; row r's 16-byte
@@ -374,10 +449,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int unit = (byte >> 4) ^ ((lane >> 1) & 3);
             if constexpr (kF32Out) {
               *reinterpret_cast<float4*>(line + (unit << 4)) = make_float4(y0, y1, y2, y3);
+              track(y0, col);
+              track(y1, col + 1);
+              track(y2, col + 2);
+              track(y3, col + 3);
             } else {
               __nv_bfloat162 h0 = __floats2bfloat162_rn(y0, y1), h1 = __floats2bfloat162_rn(y2, y3);
               *reinterpret_cast<uint2*>(line + (unit << 4) + (byte & 15)) =
                   make_uint2(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1));
+              track(__low2float(h0), col);
+              track(__high2float(h0), col + 1);
+              track(__low2float(h1), col + 2);
+              track(__high2float(h1), col + 3);
             }
           }
           fence_proxy_async_smem();
@@ -394,13 +477,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int n = n0 + part * kColsPerWarp + col;
           if (n < p.N) {
             const float y = yv(col);
-            if constexpr (kF32Out)
+            if constexpr (kF32Out) {
               static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
-            else
-              static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n] = __float2bfloat16_rn(y);
+              track(y, col);
+            } else {
+              const __nv_bfloat16 h = __float2bfloat16_rn(y);
+              static_cast<__nv_bfloat16*>(p.Y)[static_cast<size_t>(row) * p.N + n] = h;
+              track(__bfloat162float(h), col);
+            }
           }
         }
       }
+    }
+    if constexpr (kChain) {
+      // one atomic max per warp: non-negative floats order as their bit patterns
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax_next = fmaxf(amax_next, __shfl_xor_sync(0xffffffffu, amax_next, o));
+      if (lane == 0 && p.next_amax != nullptr && amax_next > 0.0f)
+        atomicMax(reinterpret_cast<unsigned int*>(p.next_amax), __float_as_uint(amax_next));
     }
     if (lane == 0) bulk_wait_all();  // every store of this warp has landed
   }
@@ -431,8 +525,8 @@ teardown:
 }  // namespace
 
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
-                              const float* lora_act, int M, void* Y, int out_dtype, const svdq_qkv_prologue* pro,
-                              cudaStream_t s) {
+                              const float* x_amax, const float* lora_act, int M, void* Y, int out_dtype,
+                              const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi, cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N;
   const int64_t m_pad = m_pad_of(M);
   CUtensorMap tm_a, tm_sfa, tm_la;
@@ -463,6 +557,10 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   p.rope_sin = pro ? pro->rope_sin : nullptr;
   p.eps = pro ? pro->eps : 0.0f;
   p.qk_cols = pro ? 2 * pro->heads * pro->head_dim : 0;
+  p.x_amax = x_amax;
+  p.g_w = w->g_w;
+  p.next_il = epi ? epi->next_inv_lambda : nullptr;
+  p.next_amax = epi ? epi->next_amax : nullptr;
   // Y through TMA stores when its rows are whole multiples of 16 bytes
   const bool f32 = out_dtype == SVDQ_OUT_F32;
   const uint64_t row_bytes = static_cast<uint64_t>(N) * (f32 ? 4 : 2);
@@ -472,8 +570,29 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
                                        N, M, row_bytes, f32 ? 16 : 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int pairs = std::min(tiles, num_sms(w->device) / 2);
-  auto kern = pro ? (f32 ? gemm_nvfp4_kernel<true, true> : gemm_nvfp4_kernel<false, true>)
-                  : (f32 ? gemm_nvfp4_kernel<true, false> : gemm_nvfp4_kernel<false, false>);
+  const int mode = pro ? kModeQkv
+                   : !epi ? kModePlain
+                   : epi->activation == SVDQ_ACT_GELU_TANH ? kModeChainGelu
+                                                          : kModeChain;
+  // the chained variants are reached through the dynamic entry points only
+  const bool dyn = x_amax != nullptr;
+  decltype(&gemm_nvfp4_kernel<false, kModePlain, false>) kern;
+  switch (mode) {
+    case kModeQkv:
+      kern = dyn ? (f32 ? gemm_nvfp4_kernel<true, kModeQkv, true> : gemm_nvfp4_kernel<false, kModeQkv, true>)
+                 : (f32 ? gemm_nvfp4_kernel<true, kModeQkv, false> : gemm_nvfp4_kernel<false, kModeQkv, false>);
+      break;
+    case kModeChain:
+      kern = f32 ? gemm_nvfp4_kernel<true, kModeChain, true> : gemm_nvfp4_kernel<false, kModeChain, true>;
+      break;
+    case kModeChainGelu:
+      kern = f32 ? gemm_nvfp4_kernel<true, kModeChainGelu, true> : gemm_nvfp4_kernel<false, kModeChainGelu, true>;
+      break;
+    default:
+      kern = dyn ? (f32 ? gemm_nvfp4_kernel<true, kModePlain, true> : gemm_nvfp4_kernel<false, kModePlain, true>)
+                 : (f32 ? gemm_nvfp4_kernel<true, kModePlain, false> : gemm_nvfp4_kernel<false, kModePlain, false>);
+  }
+  if (mode >= kModeChain && !dyn) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

@@ -73,13 +73,18 @@ cudaError_t launch_smoothing_lambda(const uint16_t* X, int M, const float* W, in
                                     float* scratch, cudaStream_t s);
 cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* lambda, const uint16_t* L1,
                            const uint16_t* L2, const uint16_t* bias, cudaStream_t s);
+cudaError_t launch_act_amax(const svdq_weights* w, const uint16_t* X, int M, float* amax, cudaStream_t s);
 cudaError_t launch_act_global_scale(const svdq_weights* w, const uint16_t* X, int M, float* g_x, cudaStream_t s);
-cudaError_t launch_quantize(const svdq_weights* w, const uint16_t* X, int M, float g_x, uint8_t* qx, void* sx,
-                            float* lora_act, cudaStream_t s);
-// `pro` (may be null): the QKV attention prologue applied in the epilogue
+// `x_amax` (may be null): the dynamic tensor scale's device amax, which
+// then replaces g_x (NVFP4)
+// `zero_word` (may be null) is set to 0 by the kernel
+cudaError_t launch_quantize(const svdq_weights* w, const uint16_t* X, int M, float g_x, const float* x_amax,
+                            uint8_t* qx, void* sx, float* lora_act, float* zero_word, cudaStream_t s);
+// `pro` (may be null): the QKV attention prologue applied in the epilogue;
+// `epi` (may be null, never with `pro`): activation and next-layer amax
 cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const uint8_t* sx, float g_x,
-                              const float* lora_act, int M, void* Y, int out_dtype, const svdq_qkv_prologue* pro,
-                              cudaStream_t s);
+                              const float* x_amax, const float* lora_act, int M, void* Y, int out_dtype,
+                              const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi, cudaStream_t s);
 size_t lowrank_workspace_bytes(int N, int K);
 cudaError_t launch_lowrank(const float* W, int N, int K, const float* lambda, int rank, int ell, int power_steps,
                            const float* omega, uint16_t* L1, uint16_t* L2, void* workspace, cudaStream_t s);

@@ -20,6 +20,8 @@ SVDQ_INT4 = 1
 SVDQ_AWQ_W4A16 = 2
 SVDQ_OUT_BF16 = 0
 SVDQ_OUT_F32 = 1
+SVDQ_ACT_NONE = 0
+SVDQ_ACT_GELU_TANH = 1
 
 STATUS_NAMES = {
     0: "SVDQ_OK",
@@ -68,6 +70,15 @@ def make_qkv_prologue(heads: int, norm_q, norm_k, rope_cos, rope_sin, eps: float
     return QkvPrologue(heads, head_dim, float(eps), _ptr(norm_q), _ptr(norm_k), _ptr(rope_cos), _ptr(rope_sin))
 
 
+class EpilogueNext(ctypes.Structure):
+    _fields_ = [("activation", ctypes.c_int32), ("next_inv_lambda", ctypes.c_void_p), ("next_amax", ctypes.c_void_p)]
+
+
+def make_epilogue_next(activation: int = SVDQ_ACT_NONE, next_inv_lambda=None, next_amax=None) -> EpilogueNext:
+    """The caller keeps the device tensors alive while the struct is used."""
+    return EpilogueNext(int(activation), _ptr(next_inv_lambda), _ptr(next_amax))
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -83,9 +94,15 @@ _SIGS = {
     "svdq_weights_destroy": (None, [_P]),
     "svdq_weights_get_view": (_I, [_P, ctypes.POINTER(WeightsView)]),
     "svdq_act_global_scale": (_I, [_P, _P, _I, _P, _P]),
+    "svdq_act_amax": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_scale_bytes": (_Z, [_P, _I]),
     "svdq_quantize_act_lora_down": (_I, [_P, _P, _I, _F, _P, _P, _P, _P]),
+    "svdq_quantize_act_lora_down_dyn": (_I, [_P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_w4a4_gemm_lora_up": (_I, [_P, _P, _P, _F, _P, _I, _P, _I, _P]),
+    "svdq_w4a4_gemm_lora_up_dyn": (_I, [_P, _P, _P, _P, _P, _I, ctypes.POINTER(QkvPrologue),
+                                        ctypes.POINTER(EpilogueNext), _P, _I, _P]),
+    "svdq_linear_forward_dyn": (_I, [_P, _P, _I, _P, ctypes.POINTER(QkvPrologue), ctypes.POINTER(EpilogueNext), _P,
+                                     _I, _P, _Z, _P]),
     "svdq_w4a4_gemm_lora_up_qkv": (_I, [_P, _P, _P, _F, _P, _I, ctypes.POINTER(QkvPrologue), _P, _I, _P]),
     "svdq_workspace_bytes": (_Z, [_P, _I]),
     "svdq_linear_forward": (_I, [_P, _P, _I, _F, _P, _I, _P, _Z, _P]),
@@ -200,6 +217,10 @@ def svdq_act_global_scale(w: Weights, X: torch.Tensor, g_x: torch.Tensor, stream
            "svdq_act_global_scale")
 
 
+def svdq_act_amax(w: Weights, X: torch.Tensor, amax: torch.Tensor, stream=None) -> None:
+    _check(load_library().svdq_act_amax(w.handle, _ptr(X), X.shape[0], _ptr(amax), _stream(stream)), "svdq_act_amax")
+
+
 def svdq_act_scale_bytes(w: Weights, M: int) -> int:
     return load_library().svdq_act_scale_bytes(w.handle, M)
 
@@ -211,6 +232,33 @@ def svdq_workspace_bytes(w: Weights, M: int) -> int:
 def svdq_quantize_act_lora_down(w: Weights, X, M: int, g_x: float, qx, sx, lora_act, stream=None) -> None:
     _check(load_library().svdq_quantize_act_lora_down(w.handle, _ptr(X), M, float(g_x), _ptr(qx), _ptr(sx),
                                                       _ptr(lora_act), _stream(stream)), "svdq_quantize_act_lora_down")
+
+
+def svdq_quantize_act_lora_down_dyn(w: Weights, X, M: int, x_amax, qx, sx, lora_act, stream=None) -> None:
+    _check(load_library().svdq_quantize_act_lora_down_dyn(w.handle, _ptr(X), M, _ptr(x_amax), _ptr(qx), _ptr(sx),
+                                                          _ptr(lora_act), _stream(stream)),
+           "svdq_quantize_act_lora_down_dyn")
+
+
+def _byref(s):
+    return None if s is None else ctypes.byref(s)
+
+
+def svdq_w4a4_gemm_lora_up_dyn(w: Weights, qx, sx, x_amax, lora_act, M: int, Y, pro: QkvPrologue | None = None,
+                               epi: EpilogueNext | None = None, out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    _check(load_library().svdq_w4a4_gemm_lora_up_dyn(w.handle, _ptr(qx), _ptr(sx), _ptr(x_amax), _ptr(lora_act), M,
+                                                     _byref(pro), _byref(epi), _ptr(Y), out_dtype, _stream(stream)),
+           "svdq_w4a4_gemm_lora_up_dyn")
+
+
+def svdq_linear_forward_dyn(w: Weights, X, M: int, x_amax, Y, workspace, ws_bytes: int,
+                            pro: QkvPrologue | None = None, epi: EpilogueNext | None = None,
+                            out_dtype: int = SVDQ_OUT_BF16, stream=None) -> None:
+    """The layer with the dynamic tensor scale; x_amax None computes it
+    from X inside the call (an amax pass into the workspace)."""
+    _check(load_library().svdq_linear_forward_dyn(w.handle, _ptr(X), M, _ptr(x_amax), _byref(pro), _byref(epi),
+                                                  _ptr(Y), out_dtype, _ptr(workspace), ws_bytes, _stream(stream)),
+           "svdq_linear_forward_dyn")
 
 
 def svdq_w4a4_gemm_lora_up(w: Weights, qx, sx, g_x: float, lora_act, M: int, Y, out_dtype: int = SVDQ_OUT_BF16,

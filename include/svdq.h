@@ -195,6 +195,14 @@ SVDQ_API svdq_status svdq_weights_get_view(const svdq_weights* w, svdq_weights_v
  * g_x [device] (one fp32).  X [device] M x K bf16, M >= 1. */
 SVDQ_API svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t* X, int32_t M, float* g_x, void* stream);
 
+/* Dynamic activation tensor scale (NVFP4): writes amax |X_hat|, X_hat =
+ * RN32(X * inv_lambda), to amax [device] (one fp32, 4-byte aligned; the
+ * call zeroes it first, then max-reduces; NaN inputs are skipped).  The
+ * _dyn entry points take such a word and use g_x = RN32(amax / 2688)
+ * (1 when amax is 0) on the device, with no host round trip: the same
+ * value svdq_act_global_scale writes.  X [device] M x K bf16, M >= 1. */
+SVDQ_API svdq_status svdq_act_amax(const svdq_weights* w, const uint16_t* X, int32_t M, float* amax, void* stream);
+
 /* Bytes of the activation scale buffer sx for M rows:
  * NVFP4: ceil(M/128)*128 * K/16 (tiled layout); INT4: 2 * K/64 * ceil(M/128)*128. */
 SVDQ_API size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M);
@@ -216,6 +224,19 @@ SVDQ_API size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M);
  * lora_act M x rank_pad fp32 (may be NULL when rank == 0). */
 SVDQ_API svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
                                         uint8_t* qx, void* sx, float* lora_act, void* stream);
+
+/* svdq_quantize_act_lora_down with the dynamic tensor scale: g_x =
+ * RN32(*x_amax / 2688) (1 when *x_amax is 0), derived on the device by the
+ * kernel with the same correctly rounded operations, so the outputs equal
+ * those of the static call given that g_x.  x_amax [device] one fp32
+ * (4-byte aligned), from svdq_act_amax or a previous layer's epilogue
+ * (svdq_epilogue_next); required for NVFP4, ignored (may be NULL) for
+ * INT4.  A derived g_x that is not finite and positive sets the status
+ * word to SVDQ_ERR_INVALID_ARG (svdq_device_status); the outputs are then
+ * unspecified. */
+SVDQ_API svdq_status svdq_quantize_act_lora_down_dyn(const svdq_weights* w, const uint16_t* X, int32_t M,
+                                                     const float* x_amax, uint8_t* qx, void* sx, float* lora_act,
+                                                     void* stream);
 
 /* 4-bit GEMM with the lora-up and the bias fused into its epilogue:
  *   NVFP4: Y = RN32(g_x * g_w) * (sum_b s_x s_w sum_{k in b} e2m1(qx) e2m1(qw)
@@ -261,7 +282,50 @@ SVDQ_API svdq_status svdq_w4a4_gemm_lora_up_qkv(const svdq_weights* w, const uin
                                        const float* lora_act, int32_t M, const svdq_qkv_prologue* pro, void* Y,
                                        int32_t out_dtype, void* stream);
 
-/* Workspace bytes of svdq_linear_forward for M rows (qx, sx, lora_act). */
+/* Activations applied in the GEMM epilogue (svdq_epilogue_next). */
+typedef enum svdq_activation {
+  SVDQ_ACT_NONE = 0,
+  SVDQ_ACT_GELU_TANH = 1 /* 0.5 y (1 + tanh(sqrt(2/pi) (y + 0.044715 y^3))) */
+} svdq_activation;
+
+/* Epilogue extras for a layer whose output is the next W4A4 layer's input
+ * (the FLUX feed-forward: up-projection, GELU, down-projection), so that
+ * the next layer's dynamic tensor scale needs no pass of its own over Y.
+ *   activation       applied to y (fp32: accumulator, lora-up and bias)
+ *                    before the one rounding to the output dtype.  The
+ *                    GELU is evaluated as y / (1 + e^(-2u)), an identity
+ *                    of the tanh form, with the hardware exp2 and
+ *                    reciprocal (relative error near 1e-6).
+ *   next_inv_lambda  [device] N fp32: 1/lambda of the next layer (whose K
+ *                    is this N), 4-byte aligned; or NULL.
+ *   next_amax        [device] one fp32, 4-byte aligned; NULL exactly when
+ *                    next_inv_lambda is.  The epilogue max-reduces
+ *                    |RN32(y_stored * next_inv_lambda[n])| over the stored
+ *                    outputs (rows < M, columns < N; NaN skipped) into it,
+ *                    so that a word that held 0 ends as the amax that
+ *                    svdq_act_amax(next layer, Y) writes.  The GEMM entry
+ *                    point leaves zeroing it to the caller; the forward
+ *                    entry point zeroes it in its quantiser kernel (no
+ *                    extra launch), and it must not be that call's x_amax.
+ * NVFP4 weights only (INT4 takes NULL or extras that ask for nothing); not
+ * combined with the QKV prologue. */
+typedef struct svdq_epilogue_next {
+  int32_t activation;
+  const float* next_inv_lambda;
+  float* next_amax;
+} svdq_epilogue_next;
+
+/* svdq_w4a4_gemm_lora_up with the dynamic tensor scale (x_amax as in
+ * svdq_quantize_act_lora_down_dyn: required for NVFP4, ignored for INT4),
+ * the optional QKV prologue `pro` [host] and the optional epilogue extras
+ * `epi` [host] (at most one of the two). */
+SVDQ_API svdq_status svdq_w4a4_gemm_lora_up_dyn(const svdq_weights* w, const uint8_t* qx, const void* sx,
+                                                const float* x_amax, const float* lora_act, int32_t M,
+                                                const svdq_qkv_prologue* pro, const svdq_epilogue_next* epi, void* Y,
+                                                int32_t out_dtype, void* stream);
+
+/* Workspace bytes of svdq_linear_forward for M rows (qx, sx, lora_act and
+ * one 1024-byte slot for the dynamic tensor scale's amax). */
 SVDQ_API size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M);
 
 /* The whole layer: svdq_quantize_act_lora_down then svdq_w4a4_gemm_lora_up
@@ -274,6 +338,16 @@ SVDQ_API svdq_status svdq_linear_forward(const svdq_weights* w, const uint16_t* 
 SVDQ_API svdq_status svdq_linear_forward_qkv(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
                                     const svdq_qkv_prologue* pro, void* Y, int32_t out_dtype, void* workspace,
                                     size_t ws_bytes, void* stream);
+
+/* The whole layer with the dynamic tensor scale: svdq_quantize_act_lora_down_dyn
+ * then svdq_w4a4_gemm_lora_up_dyn.  x_amax [device] as there, or NULL
+ * (NVFP4): then svdq_act_amax runs first, into the workspace's amax slot.
+ * `pro`, `epi` [host] as in svdq_w4a4_gemm_lora_up_dyn; the quantiser
+ * zeroes epi->next_amax, so a chain of layers can alternate two words. */
+SVDQ_API svdq_status svdq_linear_forward_dyn(const svdq_weights* w, const uint16_t* X, int32_t M,
+                                             const float* x_amax, const svdq_qkv_prologue* pro,
+                                             const svdq_epilogue_next* epi, void* Y, int32_t out_dtype,
+                                             void* workspace, size_t ws_bytes, void* stream);
 
 /* The layer forward without a caller-provided workspace.  No counterpart
  * in the pages: this exists for callers that cannot allocate device memory
@@ -313,8 +387,9 @@ SVDQ_API svdq_status svdq_awq_w4a16_forward(const svdq_weights* w, const uint16_
                                    int32_t out_dtype, void* stream);
 
 /* Synchronises `stream` and returns (then clears) the status word that the
- * GEMM kernels of this weight set write when a bounded wait runs out:
- * SVDQ_ERR_TIMEOUT, else SVDQ_OK (or SVDQ_ERR_CUDA if the sync failed). */
+ * kernels of this weight set write: SVDQ_ERR_TIMEOUT when a bounded wait
+ * ran out, SVDQ_ERR_INVALID_ARG when a dynamic tensor scale was not finite
+ * and positive, else SVDQ_OK (or SVDQ_ERR_CUDA if the sync failed). */
 SVDQ_API svdq_status svdq_device_status(const svdq_weights* w, void* stream);
 
 /* Self-test of the failure path every kernel shares (no counterpart in the

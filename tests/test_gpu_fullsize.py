@@ -168,3 +168,51 @@ def test_full_size_qkv_prologue(svdq):
                 half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(r_), 1e-30))) - 8)
                 assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
     assert svdq.svdq_device_status(w) == 0
+
+
+def test_full_size_mlp_chain(svdq):
+    """The FLUX feed-forward at full size (M=4608; up 3072 -> 12288, GELU,
+    down 12288 -> 3072; rank 32, NVFP4) with the dynamic tensor scale: the
+    up-projection's epilogue applies the GELU and max-reduces the down
+    layer's amax.  Sampled up rows against the oracle (the GELU widens the
+    bound by its Lipschitz constant 1.13); the amax word equal to the
+    separate amax pass over the stored output; the down layer on that
+    output, with the word as its scale, equal to the static layer."""
+    from oracle import chain as C
+    li_a = synth.make_layer("mlp_up", 2)
+    li_b = synth.make_layer("mlp_down", 3)
+    M, K, N = li_a.shape.M, li_a.shape.K, li_a.shape.N
+    ol_a = T.oracle_layer(li_a)
+    ol_b = T.oracle_layer(li_b)
+    wa = T.gpu_prepare(svdq, li_a, ol_a)
+    wb = T.gpu_prepare(svdq, li_b, ol_b)
+    words = torch.full((2,), 1e30, dtype=torch.float32, device="cuda")
+    il_b = T.dev_f32(ol_b.prep.inv_lam)
+    epi = svdq.make_epilogue_next(svdq.SVDQ_ACT_GELU_TANH, il_b, words[1:])
+    ws = T.aligned_empty(max(svdq.svdq_workspace_bytes(wa, M), svdq.svdq_workspace_bytes(wb, M)))
+    Ya = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    svdq.svdq_linear_forward_dyn(wa, T.dev_u16(li_a.x_bits), M, None, Ya, ws, ws.numel(), epi=epi)
+    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(wa) == 0
+    rows = np.sort(np.random.default_rng(13).choice(M, SAMPLE_ROWS, replace=False))
+    act = V.quantize_activations(li_a.x[rows], ol_a.prep, ol_a.gx)  # ol_a.gx: the dynamic scale of all of X
+    ystar = V.forward_from_codes(act, ol_a.prep, ol_a.gx)
+    ref = C.gelu_tanh(ystar)
+    y = Ya.float().cpu().numpy()[rows].astype(np.float64)
+    d = y - ref
+    rms = np.sqrt(np.mean(ystar ** 2))
+    assert np.linalg.norm(d) <= 1.13 * REL_F * np.linalg.norm(ystar)
+    half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
+    assert np.all(np.abs(d) <= 1.13 * MAX_ABS * rms + half_ulp)
+    a2 = torch.empty(1, dtype=torch.float32, device="cuda")
+    svdq.svdq_act_amax(wb, Ya.view(torch.int16), a2)
+    amax = np.float32(words[1].item())
+    assert np.float32(a2.item()) == amax and amax > 0
+    Yb = torch.empty((M, li_b.shape.N), dtype=torch.bfloat16, device="cuda")
+    svdq.svdq_linear_forward_dyn(wb, Ya.view(torch.int16), M, words[1:], Yb, ws, ws.numel())
+    Yb2 = torch.empty_like(Yb)
+    svdq.svdq_linear_forward(wb, Ya.view(torch.int16), M, float(np.float32(amax / np.float32(2688.0))), Yb2, ws,
+                             ws.numel(), 0)
+    torch.cuda.synchronize()
+    assert torch.equal(Yb, Yb2)
+    assert svdq.svdq_device_status(wb) == 0
