@@ -79,6 +79,7 @@ constexpr int kStagingPerWarp = 2048;
 constexpr int kStagingOff = kStages * kStageBytes;
 constexpr int kBiasOff = kStagingOff + kEpiWarps * kStagingPerWarp;  // 2 x 256 floats
 constexpr int kBarOff = kBiasOff + 2 * BN * 4;
+constexpr int kGxOff = kBarOff + 192;                      // dynamic variants: RN(g_x g_w)
 constexpr int kRedOff = kBarOff + 256;                     // QKV: one float per row of a head pair
 constexpr size_t kSmemBytes = kRedOff + 4 * 2 * 32 * 4 + 1024 /*align*/;
 
@@ -101,11 +102,21 @@ constexpr int kModePlain = 0, kModeQkv = 1, kModeChain = 2, kModeChainGelu = 3;
 // 0.044715 c0.  No cancellation for negative y (unlike 1 + tanh), so the
 // hardware exp2 and reciprocal keep the relative error near 1e-6.  z is
 // clamped so that 1 + 2^z stays finite.
-__device__ __forceinline__ float gelu_tanh(float y) {
-  const float z = fminf(__fmul_rn(y, __fmaf_rn(-0.10294324f, __fmul_rn(y, y), -2.3022082f)), 120.0f);
-  float e;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(z));
-  return __fdividef(y, 1.0f + e);
+// Two values at once with packed fp32 operations (each lane rounded as
+// the scalar form would be).
+__device__ __forceinline__ float2 gelu_tanh2(float2 y) {
+  const float2 t = __ffma2_rn(__fmul2_rn(y, y), make_float2(-0.10294324f, -0.10294324f),
+                              make_float2(-2.3022082f, -2.3022082f));
+  float2 z = __fmul2_rn(y, t);
+  z.x = fminf(z.x, 120.0f);
+  z.y = fminf(z.y, 120.0f);
+  float2 e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.x) : "f"(z.x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.y) : "f"(z.y));
+  const float2 d = __fadd2_rn(e, make_float2(1.0f, 1.0f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.x) : "f"(d.x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(d.y));
+  return __fmul2_rn(y, r);
 }
 
 struct GemmParams {
@@ -294,12 +305,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = (warp - 2) * 32 + lane;  // 0..511 over the epilogue warps
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t* const stg = smem + kStagingOff + (warp - 2) * kStagingPerWarp;  // a 128-byte-swizzled box
-    // RN(g_x g_w): as given, or from the device amax (kept out of a register
-    // in the static variants, which sit at the register limit)
+    // RN(g_x g_w): as given (a kernel parameter, no register), or from the
+    // device amax, published in shared memory by the first barrier and
+    // re-read where it is used (the epilogue sits at the register limit)
     float gxgw = p.gxgw;
+    const uint32_t gx_s = smem_u32(smem + kGxOff);
     if constexpr (kDyn) {
       const float a = *p.x_amax;
       gxgw = __fmul_rn(a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f), p.g_w);
+      if (et == 0) *reinterpret_cast<float*>(smem + kGxOff) = gxgw;
     }
     float amax_next = 0.0f;  // chained variant: max |y_stored / lambda'| over this thread's rows < M
     uint32_t acc_phase = 0;
@@ -412,16 +426,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the dynamic variants also compute y in place first, so that the
       // scale's register is free in the store loop
       if constexpr (kMode == kModeChainGelu) {
+        const float g = ld_shared_f32_fresh(gx_s);
+        const float2 g2 = make_float2(g, g);
 #pragma unroll
-        for (int c = 0; c < kColsPerWarp; ++c) {
-          const float y = __fadd_rn(__fmul_rn(__uint_as_float(v[c]), gxgw), bb[c]);
-          v[c] = __float_as_uint(kMode == kModeChainGelu ? gelu_tanh(y) : y);
+        for (int c = 0; c < kColsPerWarp; c += 2) {
+          const float2 b2 = *reinterpret_cast<const float2*>(bb + c);
+          const float2 y = __fadd2_rn(__fmul2_rn(make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), g2), b2);
+          const float2 o = gelu_tanh2(y);
+          v[c] = __float_as_uint(o.x);
+          v[c + 1] = __float_as_uint(o.y);
         }
       }
       // the value stored for column `col` of the warp's 64
-      auto yv = [&](int col) -> float {
+      auto yv = [&](int col, float g) -> float {
         if constexpr (kQkv || kMode == kModeChainGelu) return __uint_as_float(v[col]);
-        else return __fadd_rn(__fmul_rn(__uint_as_float(v[col]), gxgw), bb[col]);
+        else return __fadd_rn(__fmul_rn(__uint_as_float(v[col]), g), bb[col]);
+      };
+      // the scale for a group of columns: the parameter, or a fresh shared load
+      auto scale = [&]() -> float {
+        if constexpr (kDyn && !kQkv && kMode != kModeChainGelu) return ld_shared_f32_fresh(gx_s);
+        else return gxgw;
       };
       // chained variant: max |y_stored / lambda'| over the rows < M (columns
       // past N carry 1/lambda' = 0); the 1/lambda' buffer follows the bias
@@ -443,7 +467,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < kColsPerBox; j += 4) {
             const int col = pass * kColsPerBox + j;  // within the warp's columns
-            const float y0 = yv(col), y1 = yv(col + 1), y2 = yv(col + 2), y3 = yv(col + 3);
+            const float g = scale();
+            const float y0 = yv(col, g), y1 = yv(col + 1, g), y2 = yv(col + 2, g), y3 = yv(col + 3, g);
             const int byte = j * (kF32Out ? 4 : 2);  // within the box's 64-byte row
             uint8_t* line = stg + lane * 64;
             const int unit = (byte >> 4) ^ ((lane >> 1) & 3);
@@ -476,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int col = 0; col < kColsPerWarp; ++col) {
           const int n = n0 + part * kColsPerWarp + col;
           if (n < p.N) {
-            const float y = yv(col);
+            const float y = yv(col, scale());
             if constexpr (kF32Out) {
               static_cast<float*>(p.Y)[static_cast<size_t>(row) * p.N + n] = y;
               track(y, col);

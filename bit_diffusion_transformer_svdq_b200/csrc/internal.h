@@ -55,7 +55,8 @@ struct svdq_weights {
   float* inv_lambda;
   float* bias;
   int* status;    // written by the kernels when a bounded wait runs out
-  uint32_t* amax; // scratch word of the preparation pass
+  uint32_t* amax; // scratch: [0], [1] the preparation's amax and g_w; [2], [3] the activation amax
+                  // reduction (max, block count), zero between calls
   int8_t* qw8;    // INT4: n_pad x K unpacked codes (K permuted as above); NVFP4: null
   float2* swp;    // INT4: [K/64][n_pad] (s_w, -kI2FMagic * s_w); NVFP4: null
   int device;

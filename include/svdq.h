@@ -196,8 +196,11 @@ SVDQ_API svdq_status svdq_weights_get_view(const svdq_weights* w, svdq_weights_v
 SVDQ_API svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t* X, int32_t M, float* g_x, void* stream);
 
 /* Dynamic activation tensor scale (NVFP4): writes amax |X_hat|, X_hat =
- * RN32(X * inv_lambda), to amax [device] (one fp32, 4-byte aligned; the
- * call zeroes it first, then max-reduces; NaN inputs are skipped).  The
+ * RN32(X * inv_lambda), to amax [device] (one fp32, 4-byte aligned; NaN
+ * inputs are skipped).  The reduction runs in one kernel through a scratch
+ * slot of the weight storage, so calls that compute an amax on one weight
+ * set (this one, svdq_act_global_scale, svdq_linear_forward_dyn without
+ * x_amax) must not overlap on the GPU.  The
  * _dyn entry points take such a word and use g_x = RN32(amax / 2688)
  * (1 when amax is 0) on the device, with no host round trip: the same
  * value svdq_act_global_scale writes.  X [device] M x K bf16, M >= 1. */
