@@ -157,6 +157,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // programmatic dependent launch: the setup above may overlap the previous
+  // kernel; every global-memory access comes after this wait
+  grid_dep_wait();
+  if (threadIdx.x == 0) grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   uint32_t issued_mask = 0, issued_par = 0;
   uint32_t sc_mask = 0, sc_par = 0;  // scale-ring entries issued (teardown drain)
@@ -522,8 +526,18 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
                   : (f32 ? gemm_int4_kernel<true, false> : gemm_int4_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kI4Smem));
   if (e != cudaSuccess) return e;
-  kern<<<grid, kI4Threads, kI4Smem, s>>>(tm_ap, w->tm_qw8, tm_la, w->tm_l2, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kI4Threads, 1, 1);
+  cfg.dynamicSmemBytes = kI4Smem;
+  cfg.stream = s;
+  // programmatic dependent launch (the kernel waits before any memory access)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_ap, w->tm_qw8, tm_la, w->tm_l2, p);
 }
 
 }  // namespace svdq

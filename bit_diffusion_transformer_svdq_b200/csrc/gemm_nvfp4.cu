@@ -151,6 +151,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   constexpr bool kQkv = kMode == kModeQkv;
   constexpr bool kChain = kMode >= kModeChain;
+  // programmatic dependent launch: the CTA may be resident while the
+  // previous kernel drains; every global-memory access comes after this wait
+  grid_dep_wait();
+  if (threadIdx.x == 0) grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* bias_s = reinterpret_cast<float*>(smem + kBiasOff);
@@ -625,13 +629,15 @@ cudaError_t launch_gemm_nvfp4(const svdq_weights* w, const uint8_t* qx, const ui
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kern, tm_a, w->tm_qw, tm_sfa, w->tm_sw, tm_la, w->tm_l2, tm_y, p);
 }
 

@@ -355,6 +355,15 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+// Programmatic dependent launch.  grid_dep_wait: block until the grid this
+// one was launched behind has completed and its memory is visible (at once
+// when there is no such dependency); every global-memory access of a kernel
+// launched with programmatic serialization comes after it.
+// grid_dep_launch: let the next grid on the stream be scheduled (it still
+// waits for this grid's completion before touching memory).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // A shared-memory load the compiler can neither merge with another nor
 // hoist: a value re-read where it is used instead of held in a register.
 __device__ __forceinline__ float ld_shared_f32_fresh(uint32_t addr) {
