@@ -89,7 +89,7 @@ __device__ __forceinline__ uint32_t unpack_hi(uint32_t w) { return unpack_lo(w >
 
 struct I4Params {
   const __half* sx;   // [K/64][m_pad]
-  const float2* swp;  // [K/64][n_pad]
+  const float2* swp;  // [K/64][n_pad / 2] x (s_w[2j], s_w[2j+1], -magic s_w[2j], -magic s_w[2j+1])
   const float* bias;
   void* Y;
   int* status;
@@ -327,7 +327,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       const int uses = groups + (p.n_lora > 0 ? 1 : 0);
       for (int g = 0; g < uses; ++g, ++gcount) {
         float sxr = 0.0f;
-        // (s_w, -magic s_w) of two columns per entry, broadcast reads of the
+        // (s_w[c], s_w[c+1], -magic s_w[c], -magic s_w[c+1]) per float4:
+        // the two operand pairs of the packed FMA, broadcast reads of the
         // warp's private copy
         const float4* swq = reinterpret_cast<const float4*>(priv);
         if (g < groups) {
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             // columns per packed FMA
             const float2 f = make_float2(__int_as_float(static_cast<int>(P[c]) + 0x4B400000),
                                          __int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000));
-            const float2 u = __ffma2_rn(f, make_float2(t.x, t.z), make_float2(t.y, t.w));
+            const float2 u = __ffma2_rn(f, make_float2(t.x, t.y), make_float2(t.z, t.w));
             const float2 a = __ffma2_rn(u, sx2, make_float2(acc[c], acc[c + 1]));
             acc[c] = a.x;
             acc[c + 1] = a.y;

@@ -58,7 +58,7 @@ struct svdq_weights {
   uint32_t* amax; // scratch: [0], [1] the preparation's amax and g_w; [2], [3] the activation amax
                   // reduction (max, block count), zero between calls
   int8_t* qw8;    // INT4: n_pad x K unpacked codes (K permuted as above); NVFP4: null
-  float2* swp;    // INT4: [K/64][n_pad] (s_w, -kI2FMagic * s_w); NVFP4: null
+  float2* swp;    // INT4: [K/64][n_pad / 2] x (s_w[2j], s_w[2j+1], -kI2FMagic s_w[2j], -kI2FMagic s_w[2j+1]); NVFP4: null
   int device;
   CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows

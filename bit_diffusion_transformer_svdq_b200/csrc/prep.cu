@@ -148,7 +148,9 @@ __global__ void quantize_weights_kernel(const float* __restrict__ W, const float
 }
 
 // INT4 working copies: unpacked codes (K permuted within 8-value blocks,
-// rows N..n_pad zero) and the float scale pairs (s_w, -kI2FMagic s_w).
+// rows N..n_pad zero) and the float scales, per group and column pair
+// (s_w[2j], s_w[2j+1], -kI2FMagic s_w[2j], -kI2FMagic s_w[2j+1]): the two
+// operand pairs of the epilogue's packed FMA.
 __global__ void int4_unpack_kernel(const uint8_t* __restrict__ qw, const __half* __restrict__ sw, int N, int K,
                                    int64_t n_pad, int8_t* __restrict__ qw8, float2* __restrict__ swp) {
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
@@ -168,7 +170,10 @@ __global__ void int4_unpack_kernel(const uint8_t* __restrict__ qw, const __half*
   const size_t pairs = static_cast<size_t>(K / 64) * n_pad;
   if (i < pairs) {
     const float s = __half2float(sw[i]);
-    swp[i] = make_float2(s, -kI2FMagic * s);  // exact: an fp16 significand times 3 * 2^22
+    float* f = reinterpret_cast<float*>(swp);  // i = g * n_pad + n, n_pad even
+    const size_t b = 2 * (i & ~static_cast<size_t>(1)) + (i & 1);
+    f[b] = s;
+    f[b + 2] = -kI2FMagic * s;  // exact: an fp16 significand times 3 * 2^22
   }
 }
 
