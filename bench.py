@@ -241,7 +241,7 @@ def run_ours(args, li, rank, world, local_rank):
     t_step_ms = sum(a.elapsed_time(c) for a, _, c in ev) / args.steps
     t_step_ms = _allreduce_max(t_step_ms, world, dev)
     flops = 2.0 * M * N * K
-    value = world * flops / (t_step_ms * 1e-3) / 1e12
+    value = _job_tops(flops, t_step_ms, world)
 
     # ---- end to end through the C ABI with host buffers: H2D X, forward, D2H Y
     X_h = torch.from_numpy(li.x_bits.view(np.int16)).pin_memory()
@@ -299,7 +299,7 @@ def run_ours(args, li, rank, world, local_rank):
                                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"],
                                   "traffic": _traffic("quantize", os.path.join(csrc, "quantize.cu")),
                                   "algorithmic_bytes": q_bytes, "us_per_launch": tq * 1e6},
-            "e2e": {"value": world * flops / (t_e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+            "e2e": {"value": _job_tops(flops, t_e2e_ms, world), "unit": "TOPS",
                     "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": t_e2e_ms},
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
@@ -426,7 +426,7 @@ def run_stack(args, rank, world, local_rank):
     if rank == 0:
         print(json.dumps({
             "metric": "fused SVDQuant W4A4 linear effective TOPS, one denoising step of the block stack",
-            "value": world * flops / (t_ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "value": _job_tops(flops, t_ms, world), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
             "config": {"workload": f"{args.blocks} blocks x 4 linears (QKV, out, MLP up, down), M={M}, rank 32, nvfp4",
@@ -499,6 +499,12 @@ def run_awq(args, rank, world, local_rank):
                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes": nbytes, "peak_source": f"{peak_kind} hbm_gbs"},
             "gpu_launches": args.steps, "clocks": clocks}), flush=True)
+
+
+def _job_tops(ops_per_rank, t_ms_max, world):
+    """Whole-job throughput of N independent replicas (weak scaling): every
+    rank does the same work, and the job takes as long as its slowest rank."""
+    return world * ops_per_rank / (t_ms_max * 1e-3) / 1e12
 
 
 def _barrier(world):
