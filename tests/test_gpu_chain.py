@@ -255,3 +255,45 @@ def test_chain_argument_errors(svdq):
                                        ws4.data_ptr(), ws4.numel(), None) == 0
     torch.cuda.synchronize()
     assert svdq.svdq_device_status(w4) == 0
+
+
+@pytest.mark.parametrize("out_dtype", [0, 1], ids=["bf16", "f32"])
+def test_dyn_qkv_prologue_equals_static(svdq, out_dtype):
+    """The fused QKV projection with the dynamic scale (its own GEMM variant)
+    gives the static projection's output bit for bit; the static one is
+    checked against the oracle's prologue in the single-layer tests."""
+    li = synth.make_layer("qkv", 31, M=300, K=512, N=768)
+    ol = T.oracle_layer(li)
+    w = T.gpu_prepare(svdq, li, ol)
+    M, N, heads = 300, 768, 2
+    nq, nk, cs, sn = synth.qkv_prologue_inputs(M, 128, 23)
+    dq, dk, dc, ds = T.dev_f32(nq), T.dev_f32(nk), T.dev_f32(cs.T.copy()), T.dev_f32(sn.T.copy())
+    pro = svdq.make_qkv_prologue(heads, dq, dk, dc, ds, 1e-6)
+    X = T.dev_u16(li.x_bits)
+    ws = _ws(svdq, w, M)
+    Yd = _ydev(M, N, out_dtype)
+    svdq.svdq_linear_forward_dyn(w, X, M, None, Yd, ws, ws.numel(), pro=pro, out_dtype=out_dtype)
+    Ys = _ydev(M, N, out_dtype)
+    svdq.svdq_linear_forward_qkv(w, X, M, float(ol.gx), pro, Ys, ws, ws.numel(), out_dtype)
+    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(w) == 0
+    assert torch.equal(Yd, Ys)
+
+
+def test_dyn_forward_int4_ignores_the_scale_word(svdq):
+    """INT4 has no tensor scale: the dynamic forward (with or without an amax
+    word) is the static forward, bit for bit."""
+    li = synth.make_layer("int4", 9, M=260, K=512, N=384)
+    ol = T.oracle_layer(li, precision="int4")
+    w = T.gpu_prepare(svdq, li, ol, "int4")
+    M, N = 260, 384
+    X = T.dev_u16(li.x_bits)
+    ws = _ws(svdq, w, M)
+    junk = torch.full((1,), float("nan"), dtype=torch.float32, device="cuda")
+    Y0, Y1, Y2 = _ydev(M, N, 1), _ydev(M, N, 1), _ydev(M, N, 1)
+    svdq.svdq_linear_forward(w, X, M, 1.0, Y0, ws, ws.numel(), 1)
+    svdq.svdq_linear_forward_dyn(w, X, M, None, Y1, ws, ws.numel(), out_dtype=1)
+    svdq.svdq_linear_forward_dyn(w, X, M, junk, Y2, ws, ws.numel(), out_dtype=1)
+    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(w) == 0
+    assert torch.equal(Y0, Y1) and torch.equal(Y0, Y2)
