@@ -158,7 +158,12 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   __syncthreads();
   tc_fence_after();
   // programmatic dependent launch: the setup above may overlap the previous
-  // kernel; every global-memory access comes after this wait
+  // kernel; every global-memory access comes after this wait (the
+  // descriptors are kernel parameters: their fetch may start before it)
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_ap);
+    prefetch_tmap(&tm_b8);
+  }
   grid_dep_wait();
   if (threadIdx.x == 0) grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
@@ -167,10 +172,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (whole warp)
-    if (elect_one()) {
-      prefetch_tmap(&tm_ap);
-      prefetch_tmap(&tm_b8);
-    }
     int stage = 0;
     uint32_t phase = 0;
     uint32_t sc_count = 0;  // scale-ring entries issued so far

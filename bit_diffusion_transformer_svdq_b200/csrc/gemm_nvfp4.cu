@@ -153,6 +153,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr bool kChain = kMode >= kModeChain;
   // programmatic dependent launch: the CTA may be resident while the
   // previous kernel drains; every global-memory access comes after this wait
+  // (the descriptors are kernel parameters: their fetch may start before it)
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_sfa);
+    prefetch_tmap(&tm_sfb);
+  }
   grid_dep_wait();
   if (threadIdx.x == 0) grid_dep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -202,10 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (whole warp)
-    if (elect_one()) {
-      prefetch_tmap(&tm_a);
-      prefetch_tmap(&tm_b);
-    }
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = pair; tile < num_tiles; tile += num_pairs) {
