@@ -4,9 +4,9 @@ The pages state that both the weights' residual and the live activations are
 quantised to 4 bits (Nunchaku 4-bit in Diffusers, "Nunchaku und SVDQuant";
 ai2day "Was ist Nunchaku Lite"), in NVFP4 with a group of 16 or in INT4
 ("Native Ladefunktion" config block, "Hardware-Unterstuetzung").  They give
-no scale rule and no rounding mode; the rules below are this build's
-readings, written as a fixed sequence of IEEE fp32 operations so that a GPU
-can reproduce them bit for bit:
+no scale rule and no rounding mode; the rules below are readings (the
+plainest ones the pages support), written as a fixed sequence of IEEE fp32
+operations so that a GPU can reproduce them bit for bit:
 
 NVFP4, one group b of 16 values x (fp32) with a per-tensor fp32 scale g:
     amax_b = max |x|
