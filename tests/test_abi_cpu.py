@@ -59,7 +59,13 @@ def test_null_arguments_rejected_before_any_cuda_call(svdq):
     assert lib.svdq_w4a4_gemm_lora_up_qkv(None, None, None, 1.0, None, 4, ctypes.byref(pro), None, 0, None) == 1
     assert lib.svdq_w4a4_gemm_lora_up_qkv(None, None, None, 1.0, None, 4, None, None, 0, None) == 1
     assert lib.svdq_linear_forward_qkv(None, None, 4, 1.0, ctypes.byref(pro), None, 0, None, 0, None) == 1
-    import ctypes
+    # the dynamic-scale and chained entry points
+    epi = svdq.EpilogueNext()
+    assert lib.svdq_act_amax(None, None, 4, None, None) == 1
+    assert lib.svdq_quantize_act_lora_down_dyn(None, None, 4, None, None, None, None, None) == 1
+    assert lib.svdq_w4a4_gemm_lora_up_dyn(None, None, None, None, None, 4, None, ctypes.byref(epi), None, 0, None) == 1
+    assert lib.svdq_linear_forward_dyn(None, None, 4, None, None, ctypes.byref(epi), None, 0, None, 0, None) == 1
+    assert lib.svdq_awq_w4a16_forward(None, None, 1, None, 0, None) == 1
     out = ctypes.c_void_p()
     d = svdq.make_desc(256, 256, 16)
     assert lib.svdq_prepare_weights(ctypes.byref(d), None, None, None, None, None, None, 0, ctypes.byref(out), None) == 1
