@@ -30,6 +30,23 @@ def test_every_declared_symbol_is_exported(svdq):
     assert set(names) <= set(svdq._SIGS), set(names) - set(svdq._SIGS)
 
 
+def _prototypes():
+    """name -> number of parameters, from every SVDQ_API declaration."""
+    hdr = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    out = {}
+    for m in re.finditer(r"^SVDQ_API [^;(]*?\b(svdq_\w+)\s*\(([^;]*?)\)\s*;", hdr, re.M | re.S):
+        params = " ".join(m.group(2).split())
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_bindings_match_the_header_prototypes(svdq):
+    protos = _prototypes()
+    assert set(protos) == set(_declared())
+    for name, n in protos.items():
+        assert len(svdq._SIGS[name][1]) == n, (name, n, len(svdq._SIGS[name][1]))
+
+
 def test_status_strings(svdq):
     for code in range(8):
         assert svdq.svdq_status_string(code)
