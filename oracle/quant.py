@@ -45,6 +45,20 @@ def nvfp4_tensor_scale(amax) -> np.float32:
     return np.float32(amax / np.float32(2688.0))
 
 
+# Rows are independent, so the quantisers work through them in blocks of
+# this many rows (keeps the temporaries small; the arithmetic per element is
+# the same as on the whole matrix at once).
+_ROW_BLOCK = 256
+
+
+def _by_row_blocks(fn, x: np.ndarray):
+    R = x.shape[0]
+    if R <= _ROW_BLOCK:
+        return fn(x)
+    parts = [fn(x[i:i + _ROW_BLOCK]) for i in range(0, R, _ROW_BLOCK)]
+    return tuple(np.concatenate([p[j] for p in parts], axis=0) for j in range(len(parts[0])))
+
+
 def nvfp4_quantize(x: np.ndarray, g) -> tuple[np.ndarray, np.ndarray]:
     """Quantise rows of fp32 values, groups of 16 along the last axis.
 
@@ -53,9 +67,13 @@ def nvfp4_quantize(x: np.ndarray, g) -> tuple[np.ndarray, np.ndarray]:
     """
     x = np.asarray(x, dtype=np.float32)
     g = np.float32(g)
-    R, K = x.shape
-    if K % NVFP4_GROUP:
+    if x.shape[1] % NVFP4_GROUP:
         raise ValueError("K must be a multiple of 16")
+    return _by_row_blocks(lambda xb: _nvfp4_rows(xb, g), x)
+
+
+def _nvfp4_rows(x: np.ndarray, g: np.float32) -> tuple[np.ndarray, np.ndarray]:
+    R, K = x.shape
     xg = x.reshape(R, K // NVFP4_GROUP, NVFP4_GROUP)
     amax = np.max(np.abs(xg), axis=2)  # fp32, exact
     s_f = (amax / np.float32(6.0)) / g  # two fp32 divisions, each RN
@@ -72,9 +90,12 @@ def nvfp4_quantize(x: np.ndarray, g) -> tuple[np.ndarray, np.ndarray]:
 def nvfp4_dequantize(codes: np.ndarray, scale_bytes: np.ndarray, g) -> np.ndarray:
     """fp64 values e2m1(code) * s * g (exact products)."""
     R, K = codes.shape
-    e = F.e2m1_decode(codes).reshape(R, K // NVFP4_GROUP, NVFP4_GROUP)
-    s = F.e4m3_decode(scale_bytes)
-    return (e * s[:, :, None]).reshape(R, K) * float(np.float32(g))
+    out = np.empty((R, K), np.float64)
+    for i in range(0, R, _ROW_BLOCK):
+        e = F.e2m1_decode(codes[i:i + _ROW_BLOCK]).reshape(-1, K // NVFP4_GROUP, NVFP4_GROUP)
+        s = F.e4m3_decode(scale_bytes[i:i + _ROW_BLOCK])
+        out[i:i + _ROW_BLOCK] = (e * s[:, :, None]).reshape(-1, K) * float(np.float32(g))
+    return out
 
 
 def int4_quantize(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
@@ -84,9 +105,13 @@ def int4_quantize(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     per group).
     """
     x = np.asarray(x, dtype=np.float32)
-    R, K = x.shape
-    if K % INT4_GROUP:
+    if x.shape[1] % INT4_GROUP:
         raise ValueError("K must be a multiple of 64")
+    return _by_row_blocks(_int4_rows, x)
+
+
+def _int4_rows(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    R, K = x.shape
     xg = x.reshape(R, K // INT4_GROUP, INT4_GROUP)
     amax = np.max(np.abs(xg), axis=2)
     s_h = F.fp16_rn((amax / np.float32(7.0)).astype(np.float64))  # fp64 values on the fp16 grid

@@ -45,8 +45,9 @@ from .svd import truncated_svd
 
 def smoothing_lambda(x: np.ndarray, w: np.ndarray) -> np.ndarray:
     """Per-input-channel smoothing factor lambda (K,) in fp32."""
-    ax = np.max(np.abs(np.asarray(x, dtype=np.float64)), axis=0)
-    aw = np.max(np.abs(np.asarray(w, dtype=np.float64)), axis=0)
+    # maxima of magnitudes are exact in the inputs' own type; ratio and root in fp64
+    ax = np.max(np.abs(np.asarray(x)), axis=0).astype(np.float64)
+    aw = np.max(np.abs(np.asarray(w)), axis=0).astype(np.float64)
     with np.errstate(divide="ignore", invalid="ignore"):
         lam = np.sqrt(ax / aw)
     lam = np.where((ax == 0) | (aw == 0), 1.0, lam)
@@ -80,12 +81,19 @@ def lowrank_factors(w: np.ndarray, lam: np.ndarray, rank: int, omega: np.ndarray
 
 def residual(wt: np.ndarray, L1: np.ndarray, L2: np.ndarray) -> np.ndarray:
     """R = RN32(fp64 chain W_til - sum_t L1[t,:] L2[:,t]) in fixed t order."""
-    acc = np.asarray(wt, dtype=np.float32).astype(np.float64)
+    wt = np.asarray(wt, dtype=np.float32)
     L1d = np.asarray(L1, dtype=np.float64)
     L2d = np.asarray(L2, dtype=np.float64)
-    for t in range(L1d.shape[0]):
-        acc -= L2d[:, t:t + 1] * L1d[t:t + 1, :]
-    return acc.astype(np.float32)
+    out = np.empty(wt.shape, np.float32)
+    B = 64  # rows per block: the chain of each element is the same, blocks only keep it in cache
+    for i in range(0, wt.shape[0], B):
+        acc = wt[i:i + B].astype(np.float64)
+        tmp = np.empty_like(acc)
+        for t in range(L1d.shape[0]):
+            np.multiply(L2d[i:i + B, t:t + 1], L1d[t:t + 1, :], out=tmp)  # exact: two bf16 values
+            acc -= tmp
+        out[i:i + B] = acc
+    return out
 
 
 @dataclasses.dataclass

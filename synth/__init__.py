@@ -37,10 +37,14 @@ def bf16_bits_from_f32(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bf16 (ties to even) and return the
     16-bit patterns.  Used only to store generated inputs in bf16."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> np.uint64(16)) & np.uint64(1)
-    r = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
-    return r.astype(np.uint16)
+    flat = a.reshape(-1)
+    out = np.empty(flat.shape, np.uint16)
+    step = 1 << 20  # blocks of a million values keep the temporaries in cache
+    for i in range(0, flat.size, step):
+        u = flat[i:i + step].view(np.uint32).astype(np.uint64)
+        lsb = (u >> np.uint64(16)) & np.uint64(1)
+        out[i:i + step] = (u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)
+    return out.reshape(a.shape)
 
 
 def f32_from_bf16_bits(b: np.ndarray) -> np.ndarray:
