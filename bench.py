@@ -1,19 +1,30 @@
 """Benchmark of the SVDQuant W4A4 linear layer on B200.
 
-One step = the whole hot path on one batch: smoothing + NVFP4 activation
-quantisation + lora-down (one kernel), then the block-scaled 4-bit GEMM with
-the lora-up and bias in its epilogue (one kernel), on the FLUX-shaped fused
-QKV projection (M=4608 tokens, K=3072, N=9216, rank 32, NVFP4).
+One step = the whole hot path over one batch, for every linear of the
+workload: smoothing + 4-bit activation quantisation + lora-down (one
+kernel), then the 4-bit GEMM with the lora-up and bias in its epilogue (one
+kernel).  Workloads (--workload):
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  mlp   (default) the FLUX-shaped MLP pair: up 4608 x 3072 -> 12288, then
+        down 4608 x 12288 -> 3072 on a GELU(tanh) input, rank 32, NVFP4
+  qkv   the FLUX-shaped fused QKV projection 4608 x 3072 -> 9216, rank 32,
+        NVFP4 (--qkv-prologue adds the attention prologue to the GEMM)
+  int4  the INT4 group-64 variant on a batch of four images:
+        18432 x 3072 -> 3072, rank 32
+  tiny  64 x 256 -> 256, rank 16, NVFP4 (launch-bound; microseconds only)
+  stack one denoising step of the 57-block stack (run_stack)
+  awq   the awq_w4a16 modulation projection (run_awq)
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ...]
 
 Prints one JSON line (rank 0).  `value` is effective TOPS (2*M*N*K dense-
-equivalent operations per second, the low-rank flops not counted) summed
-over all ranks; ranks run independent replicas (the layer has no exchange
-step).  L2 is flushed before every timed step by reading a 256 MiB buffer (a read
-leaves only clean lines, so the step pays no write-back of the flush),
-outside the step's CUDA-event bracket.  `--impl reference` times the CPU oracle on the
-host cores on a bounded row sample of the same workload.
+equivalent operations per second over the step's linears, the low-rank
+flops not counted) summed over all ranks; ranks run independent replicas
+(the layer has no exchange step).  L2 is flushed before every timed step by
+reading a 256 MiB buffer (a read leaves only clean lines, so the step pays
+no write-back of the flush), outside the step's CUDA-event bracket.
+`--impl reference` times the CPU oracle on the host cores on a bounded row
+sample of the same workload.
 """
 from __future__ import annotations
 
@@ -32,8 +43,16 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "qkv"
-SEED = 2
+# workload -> (description, [(layer shape, seed), ...])
+LAYER_WORKLOADS = {
+    "mlp": ("FLUX MLP pair: up 4608x3072->12288 then down 4608x12288->3072 (GELU(tanh) input), rank 32, nvfp4",
+            [("mlp_up", 2), ("mlp_down", 3)]),
+    "qkv": ("FLUX fused QKV projection 4608x3072->9216, rank 32, nvfp4", [("qkv", 2)]),
+    "int4": ("INT4 group-64, four images: 18432x3072->3072, rank 32", [("int4", 4)]),
+    "tiny": ("tiny 64x256->256, rank 16, nvfp4", [("tiny", 1)]),
+}
+CPU_SAMPLE_ROWS = 128
+METRIC = "fused SVDQuant W4A4 linear effective TOPS"
 
 
 def _peaks():
@@ -48,13 +67,13 @@ def _src_hash(path):
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
 
-def _traffic(kernel_key, src):
+def _traffic(key, src):
     """dram bytes per launch from the committed ncu summary, or None if the
     kernel source changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p)).get(kernel_key)
+    d = json.load(open(p)).get(key)
     if not d or d.get("src_sha") != _src_hash(src):
         return None
     return d.get("dram_bytes_per_launch")
@@ -73,6 +92,8 @@ class ClockSampler:
         self.proc = None
 
     def start(self):
+        """Starts sampling and returns once the first sample has arrived (at
+        most 3 s), so that the timed region that follows is covered."""
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
                                           "-lms", "20", "-i", self.gpu], stdout=subprocess.PIPE,
@@ -81,6 +102,10 @@ class ClockSampler:
             self.t.start()
         except OSError:
             self.proc = None
+            return
+        t_end = time.time() + 3.0
+        while not self.rows and time.time() < t_end:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -89,6 +114,9 @@ class ClockSampler:
     def stop(self, t0, t1):
         if not self.proc:
             return None
+        t_end = time.time() + 0.5  # one sample past the timed region
+        while not any(ts > t1 for ts, _ in self.rows) and time.time() < t_end:
+            time.sleep(0.01)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -105,21 +133,33 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sel)}
 
 
-def _oracle_sample(li, rows, reps=1):
-    """Times the oracle (as it stands) on `rows` rows: quantise + lora-down +
-    fp64 forward.  Weight preparation is done first and not timed."""
+def _sampler(local_rank):
+    return ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ
+                        else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+
+
+def _oracle_prepare(li):
+    """Oracle weight preparation of one layer (untimed)."""
     from oracle import svdq as V
     lam = V.smoothing_lambda(li.x, li.w)
     L1, L2 = V.lowrank_factors(li.w, lam, li.shape.rank)
-    prep = V.prepare_weights(li.w, lam, L1, L2, li.bias)
-    gx = V.act_global_scale(li.x, prep.inv_lam)
-    xs = li.x[:rows]
-    times = []
-    for _ in range(reps):
-        t = time.perf_counter()
-        V.forward(xs, prep, gx)
-        times.append(time.perf_counter() - t)
-    return times
+    prep = V.prepare_weights(li.w, lam, L1, L2, li.bias, li.shape.precision)
+    gx = V.act_global_scale(li.x, prep.inv_lam) if li.shape.precision == "nvfp4" else None
+    return prep, gx
+
+
+def _oracle_step(lis, preps, rows):
+    """One bounded-sample step of the oracle as it stands: quantise +
+    lora-down + fp64 forward of `rows` rows of every layer.  Returns
+    (seconds, operations counted like the GPU metric)."""
+    from oracle import svdq as V
+    t = time.perf_counter()
+    ops = 0.0
+    for li, (prep, gx) in zip(lis, preps):
+        r = min(rows, li.shape.M)
+        V.forward(li.x[:r], prep, gx)
+        ops += 2.0 * r * li.shape.N * li.shape.K
+    return time.perf_counter() - t, ops
 
 
 def _cpu_threads():
@@ -131,186 +171,229 @@ def _cpu_threads():
         return os.cpu_count() or 1
 
 
-def run_reference(args, li, rank, world):
+def _layer_inputs(args):
+    import synth
+    desc, specs = LAYER_WORKLOADS[args.workload]
+    over = {"M": args.rows} if args.rows else {}
+    return desc, [synth.make_layer(name, seed, **over) for name, seed in specs]
+
+
+def run_reference(args, rank, world):
     if rank != 0:
         return
-    K, N = li.shape.K, li.shape.N
-    rows = 128
-    times = _oracle_sample(li, rows, reps=args.warmup + args.steps)[args.warmup:]
-    t = sum(times) / len(times)
-    value = 2.0 * rows * N * K / t / 1e12
+    desc, lis = _layer_inputs(args)
+    preps = [_oracle_prepare(li) for li in lis]
+    res = [_oracle_step(lis, preps, CPU_SAMPLE_ROWS) for _ in range(args.warmup + args.steps)][args.warmup:]
+    t = sum(r[0] for r in res) / len(res)
+    value = res[0][1] / t / 1e12
+    rows = min(CPU_SAMPLE_ROWS, lis[0].shape.M)
+    sample = f"{rows} rows of each of the {len(lis)} linear(s) per step, numpy fp64 oracle, weights prepared untimed"
     line = {
-        "impl": "reference", "metric": "fused SVDQuant W4A4 linear effective TOPS", "value": value, "unit": "TOPS",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD} M={li.shape.M} K={K} N={N} rank={li.shape.rank} nvfp4",
-                   "sample_rows_per_step": rows},
-        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": _cpu_threads(), "kind": "oracle",
-                         "sample": f"{rows} of {li.shape.M} rows per step, numpy fp64 oracle"},
+        "config": {"workload": f"{args.workload}: {desc}", "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": _cpu_threads(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, li, rank, world, local_rank):
+def _gpu_layer(svdq, li, dev, seed):
+    """Offline preparation on the GPU (untimed): smoothing factor, the
+    library's factoriser from a seeded start block, weight preparation and
+    the calibrated activation tensor scale."""
     import torch
     import synth
+    M, K, N, r = li.shape.M, li.shape.K, li.shape.N, li.shape.rank
+    X = torch.from_numpy(li.x_bits.view(np.int16)).to(dev)
+    W = torch.from_numpy(li.w).to(dev)
+    bias = torch.from_numpy(li.bias_bits.view(np.int16)).to(dev)
+    lam = torch.empty(K, dtype=torch.float32, device=dev)
+    svdq.svdq_smoothing_lambda(X, W, lam, torch.empty(2 * K, dtype=torch.float32, device=dev))
+    L1 = torch.empty((r, K), dtype=torch.int16, device=dev)
+    L2 = torch.empty((N, r), dtype=torch.int16, device=dev)
+    omega = torch.from_numpy(synth.svd_start_block(N, r + 16, seed)).to(dev)
+    lr_ws = svdq.alloc_workspace(None, 0, dev, nbytes=svdq.svdq_lowrank_workspace_bytes(N, K))
+    svdq.svdq_lowrank_factors(W, lam, r, omega, L1, L2, lr_ws)
+    prec = svdq.SVDQ_INT4 if li.shape.precision == "int4" else svdq.SVDQ_NVFP4
+    w = svdq.prepare_layer(W, lam, L1, L2, bias, r, prec)
+    gx = 1.0
+    if prec == svdq.SVDQ_NVFP4:
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+        svdq.svdq_act_global_scale(w, X, g)
+        gx = float(g.item())
+    ws = svdq.alloc_workspace(w, M, dev)
+    sx_off = (M * K // 2 + 1023) // 1024 * 1024
+    la_off = sx_off + (svdq.svdq_act_scale_bytes(w, M) + 1023) // 1024 * 1024
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    act_scale_bytes = M * K // 16 if prec == svdq.SVDQ_NVFP4 else M * (K // 64) * 2
+    q_bytes = M * K * 2 + M * K // 2 + act_scale_bytes + M * w.view().rank_pad * 4
+    return dict(name=li.shape.name, w=w, X=X, gx=gx, M=M, K=K, N=N, prec=prec, qx=ws, sx=ws[sx_off:],
+                la=ws[la_off:], Y=Y, flops=2.0 * M * N * K, q_bytes=q_bytes)
+
+
+def run_layers(args, rank, world, local_rank):
+    import torch
     from bit_diffusion_transformer_svdq_b200 import svdq
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     svdq.load_library()
-    M, K, N, r = li.shape.M, li.shape.K, li.shape.N, li.shape.rank
     stream = torch.cuda.current_stream()
-
-    # ---- offline preparation (untimed): calibration, factorisation, weight prep
-    X = torch.from_numpy(li.x_bits.view(np.int16)).to(dev)
-    W = torch.from_numpy(li.w).to(dev)
-    bias = torch.from_numpy(li.bias_bits.view(np.int16)).to(dev)
-    lam = torch.empty(K, dtype=torch.float32, device=dev)
-    scratch = torch.empty(2 * K, dtype=torch.float32, device=dev)
-    svdq.svdq_smoothing_lambda(X, W, lam, scratch)
-    # the offline factoriser: rank-r factors of W_til^T by the library's
-    # GPU subspace iteration from a seeded start block
-    L1 = torch.empty((r, K), dtype=torch.int16, device=dev)
-    L2 = torch.empty((N, r), dtype=torch.int16, device=dev)
-    omega = torch.from_numpy(synth.svd_start_block(N, r + 16, SEED)).to(dev)
-    lr_ws = svdq.alloc_workspace(None, 0, dev, nbytes=svdq.svdq_lowrank_workspace_bytes(N, K))
-    svdq.svdq_lowrank_factors(W, lam, r, omega, L1, L2, lr_ws)
-    del lr_ws, omega
-    w = svdq.prepare_layer(W, lam, L1, L2, bias, r)
-    gx_t = torch.empty(1, dtype=torch.float32, device=dev)
-    svdq.svdq_act_global_scale(w, X, gx_t)
-    gx = float(gx_t.item())
-    del W
-
-    ws = svdq.alloc_workspace(w, M, dev)
-    qx = ws
-    sx_off = (M * K // 2 + 1023) // 1024 * 1024
-    sx = ws[sx_off:]
-    la_off = sx_off + (svdq.svdq_act_scale_bytes(w, M) + 1023) // 1024 * 1024
-    la = ws[la_off:]
-    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    desc, lis = _layer_inputs(args)
+    _, specs = LAYER_WORKLOADS[args.workload]
+    layers = [_gpu_layer(svdq, li, dev, seed) for li, (_, seed) in zip(lis, specs)]
     flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
     pro = None
     if args.qkv_prologue:  # the fused attention prologue: seeded QK-norm weights and rotary tables
-        nq, nk, cs, sn = synth.qkv_prologue_inputs(M, 128, SEED)
+        if args.workload != "qkv":
+            raise SystemExit("--qkv-prologue needs --workload qkv")
+        import synth
+        L = layers[0]
+        nq, nk, cs, sn = synth.qkv_prologue_inputs(L["M"], 128, 2)
         pro_t = [torch.from_numpy(a).to(dev) for a in (nq, nk, cs.T.copy(), sn.T.copy())]
-        pro = svdq.make_qkv_prologue(N // 384, *pro_t, eps=1e-6)
+        pro = svdq.make_qkv_prologue(L["N"] // 384, *pro_t, eps=1e-6)
 
-    def gemm():
+    def quantize(L):
+        svdq.svdq_quantize_act_lora_down(L["w"], L["X"], L["M"], L["gx"], L["qx"], L["sx"], L["la"], stream)
+
+    def gemm(L):
         if pro is None:
-            svdq.svdq_w4a4_gemm_lora_up(w, qx, sx, gx, la, M, Y, svdq.SVDQ_OUT_BF16, stream)
+            svdq.svdq_w4a4_gemm_lora_up(L["w"], L["qx"], L["sx"], L["gx"], L["la"], L["M"], L["Y"],
+                                        svdq.SVDQ_OUT_BF16, stream)
         else:
-            svdq.svdq_w4a4_gemm_lora_up_qkv(w, qx, sx, gx, la, M, pro, Y, svdq.SVDQ_OUT_BF16, stream)
-
-    def step():
-        svdq.svdq_quantize_act_lora_down(w, X, M, gx, qx, sx, la, stream)
-        gemm()
+            svdq.svdq_w4a4_gemm_lora_up_qkv(L["w"], L["qx"], L["sx"], L["gx"], L["la"], L["M"], pro, L["Y"],
+                                            svdq.SVDQ_OUT_BF16, stream)
 
     for _ in range(args.warmup):
         flush.sum()
-        step()
+        for L in layers:
+            quantize(L)
+            gemm(L)
     torch.cuda.synchronize()
-    assert svdq.svdq_device_status(w) == 0
+    assert all(svdq.svdq_device_status(L["w"]) == 0 for L in layers)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    nl = len(layers)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 * nl + 1)] for _ in range(args.steps)]
+    sampler = _sampler(local_rank)
     sampler.start()
-    time.sleep(0.1)
     _barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
     for i in range(args.steps):
         flush.sum()
-        e0, e1, e2 = ev[i]
-        e0.record(stream)
-        svdq.svdq_quantize_act_lora_down(w, X, M, gx, qx, sx, la, stream)
-        e1.record(stream)
-        gemm()
-        e2.record(stream)
+        ev[i][0].record(stream)
+        for j, L in enumerate(layers):
+            quantize(L)
+            ev[i][2 * j + 1].record(stream)
+            gemm(L)
+            ev[i][2 * j + 2].record(stream)
     torch.cuda.synchronize()
     _barrier(world)
     t_wall1 = time.time()
     clocks = sampler.stop(t_wall0, t_wall1)
-    assert svdq.svdq_device_status(w) == 0
+    assert all(svdq.svdq_device_status(L["w"]) == 0 for L in layers)
 
-    t_q = [a.elapsed_time(b) for a, b, _ in ev]
-    t_g = [b.elapsed_time(c) for _, b, c in ev]
-    t_step_ms = sum(a.elapsed_time(c) for a, _, c in ev) / args.steps
-    t_step_ms = _allreduce_max(t_step_ms, world, dev)
-    flops = 2.0 * M * N * K
+    # per layer: mean quantiser and GEMM times (seconds) over the timed steps
+    tq = [statistics.mean(e[2 * j].elapsed_time(e[2 * j + 1]) for e in ev) * 1e-3 for j in range(nl)]
+    tg = [statistics.mean(e[2 * j + 1].elapsed_time(e[2 * j + 2]) for e in ev) * 1e-3 for j in range(nl)]
+    t_step_ms = _allreduce_max(statistics.mean(e[0].elapsed_time(e[-1]) for e in ev), world, dev)
+    flops = sum(L["flops"] for L in layers)
     value = _job_tops(flops, t_step_ms, world)
 
-    # ---- end to end through the C ABI with host buffers: H2D X, forward, D2H Y
-    X_h = torch.from_numpy(li.x_bits.view(np.int16)).pin_memory()
-    Y_h = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
-    X_d = torch.empty_like(X)
-    ws2 = svdq.alloc_workspace(w, M, dev)
-    e2e_steps = max(3, min(args.steps, 20))
-    def forward():
-        if pro is None:
-            svdq.svdq_linear_forward(w, X_d, M, gx, Y, ws2, ws2.numel(), svdq.SVDQ_OUT_BF16, stream)
-        else:
-            svdq.svdq_linear_forward_qkv(w, X_d, M, gx, pro, Y, ws2, ws2.numel(), svdq.SVDQ_OUT_BF16, stream)
+    # ---- end to end through the C ABI with host buffers: H2D X, the layer
+    # forward (svdq_linear_forward), D2H Y, for every linear of the step
+    host = [(torch.from_numpy(li.x_bits.view(np.int16)).pin_memory(),
+             torch.empty((L["M"], L["N"]), dtype=torch.bfloat16).pin_memory(), torch.empty_like(L["X"]),
+             svdq.alloc_workspace(L["w"], L["M"], dev)) for li, L in zip(lis, layers)]
 
+    def e2e_step():
+        for (X_h, Y_h, X_d, ws), L in zip(host, layers):
+            X_d.copy_(X_h, non_blocking=True)
+            if pro is None:
+                svdq.svdq_linear_forward(L["w"], X_d, L["M"], L["gx"], L["Y"], ws, ws.numel(), svdq.SVDQ_OUT_BF16,
+                                         stream)
+            else:
+                svdq.svdq_linear_forward_qkv(L["w"], X_d, L["M"], L["gx"], pro, L["Y"], ws, ws.numel(),
+                                             svdq.SVDQ_OUT_BF16, stream)
+            Y_h.copy_(L["Y"], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
     for _ in range(2):
-        X_d.copy_(X_h, non_blocking=True)
-        forward()
-        Y_h.copy_(Y, non_blocking=True)
+        e2e_step()
     torch.cuda.synchronize()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s0.record(stream)
     for _ in range(e2e_steps):
-        X_d.copy_(X_h, non_blocking=True)
-        forward()
-        Y_h.copy_(Y, non_blocking=True)
+        e2e_step()
     s1.record(stream)
     torch.cuda.synchronize()
     t_e2e_ms = _allreduce_max(s0.elapsed_time(s1) / e2e_steps, world, dev)
 
     peaks, peak_kind = _peaks()
-    fp4_peak = peaks["bf16_tflops"] * 4.0  # nominal dense FP4 / BF16 ratio (9 / 2.25)
-    tg = statistics.mean(t_g) * 1e-3
-    tq = statistics.mean(t_q) * 1e-3
-    gemm_tflops = flops / tg / 1e12
-    q_bytes = M * K * 2 + M * K // 2 + M * K // 16 + M * w.view().rank_pad * 4
-    q_gbs = q_bytes / tq / 1e9
     csrc = os.path.join(ROOT, "bit_diffusion_transformer_svdq_b200", "csrc")
+    kernels = []
+    for j, L in enumerate(layers):
+        int4 = L["prec"] == svdq.SVDQ_INT4
+        # nominal dense ratios to bf16: FP4 9 / 2.25 = 4, INT8 4.5 / 2.25 = 2
+        peak = peaks["bf16_tflops"] * (2.0 if int4 else 4.0)
+        gk = "gemm_int4_kernel" if int4 else "gemm_nvfp4_kernel"
+        tkey = f"{'gemm_int4' if int4 else 'gemm_nvfp4'}/{L['name']}"
+        kernels.append({"kernel": gk, "layer": L["name"], "bound": "tensor", "us_per_launch": tg[j] * 1e6,
+                        "achieved": L["flops"] / tg[j] / 1e12, "peak": peak, "unit": "TFLOP/s",
+                        "frac": L["flops"] / tg[j] / 1e12 / peak,
+                        "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                                       f"{2 if int4 else 4} (nominal {'INT8' if int4 else 'FP4'}:BF16)",
+                        "traffic": _traffic(tkey, os.path.join(csrc, "gemm_int4.cu" if int4 else "gemm_nvfp4.cu"))})
+        kernels.append({"kernel": "quantize_lora_down_kernel", "layer": L["name"], "bound": "hbm",
+                        "us_per_launch": tq[j] * 1e6, "achieved": L["q_bytes"] / tq[j] / 1e9,
+                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": L["q_bytes"] / tq[j] / 1e9 / peaks["hbm_gbs"], "algorithmic_bytes": L["q_bytes"],
+                        "traffic": _traffic(f"quantize/{L['name']}", os.path.join(csrc, "quantize.cu"))})
+    gemms = [k for k in kernels if k["bound"] == "tensor"]
+    quants = [k for k in kernels if k["bound"] == "hbm"]
+    # the dominant kernel: the GEMM (every layer's launch of it, averaged)
+    g_us = statistics.mean(k["us_per_launch"] for k in gemms)
+    g_flops = statistics.mean(L["flops"] for L in layers)
+    roof = {"bound": "tensor", "kernel": gemms[0]["kernel"], "achieved": g_flops / g_us / 1e6, "peak": gemms[0]["peak"],
+            "unit": "TFLOP/s", "frac": g_flops / g_us / 1e6 / gemms[0]["peak"],
+            "traffic": (statistics.mean(k["traffic"] for k in gemms) if all(k["traffic"] for k in gemms) else None),
+            "peak_source": gemms[0]["peak_source"], "us_per_launch": g_us,
+            "launches_per_step": len(gemms)}
+    q_big = max(quants, key=lambda k: k["algorithmic_bytes"])  # the largest activation pass
+    roof_q = {k: q_big[k] for k in ("bound", "kernel", "layer", "achieved", "peak", "unit", "frac", "traffic",
+                                    "algorithmic_bytes", "us_per_launch")}
 
     if rank == 0:
         line = {
-            "metric": "fused SVDQuant W4A4 linear effective TOPS"
-                      + (" (QKV projection with the fused attention prologue)" if pro is not None else ""),
+            "metric": METRIC + (" (QKV projection with the fused attention prologue)" if pro is not None else ""),
             "value": value, "unit": "TOPS",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4" if layers[0]["prec"] == svdq.SVDQ_INT4 else "nvfp4",
             "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD} M={M} K={K} N={N} rank={r} nvfp4 (FLUX fused QKV projection)",
+            "config": {"workload": f"{args.workload}: {desc}",
+                       "linears": [f"{L['name']} M={L['M']} K={L['K']} N={L['N']}" for L in layers],
                        "l2": "flushed (256 MiB read) before each step, outside the step's event bracket",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "tensor", "kernel": "gemm_nvfp4_kernel", "achieved": gemm_tflops, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak,
-                         "traffic": _traffic("gemm_nvfp4", os.path.join(csrc, "gemm_nvfp4.cu")),
-                         "peak_source": f"{peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s x 4 (nominal FP4:BF16)",
-                         "us_per_launch": tg * 1e6},
-            "roofline_quantize": {"bound": "hbm", "kernel": "quantize_lora_down_kernel", "achieved": q_gbs,
-                                  "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"],
-                                  "traffic": _traffic("quantize", os.path.join(csrc, "quantize.cu")),
-                                  "algorithmic_bytes": q_bytes, "us_per_launch": tq * 1e6},
+            "roofline": roof,
+            "roofline_quantize": roof_q,
+            "kernels": kernels,
             "e2e": {"value": _job_tops(flops, t_e2e_ms, world), "unit": "TOPS",
-                    "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2, "ms_per_step": t_e2e_ms},
-            "gpu_launches": 2 * args.steps,
+                    "h2d_bytes_per_step": sum(L["M"] * L["K"] * 2 for L in layers),
+                    "d2h_bytes_per_step": sum(L["M"] * L["N"] * 2 for L in layers), "ms_per_step": t_e2e_ms},
+            "gpu_launches": 2 * nl * args.steps,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            rows = 128
-            times = _oracle_sample(li, rows, reps=2)
-            t = min(times)
-            line["cpu_baseline"] = {"value": 2.0 * rows * N * K / t / 1e12, "unit": "TOPS", "cores": _cpu_threads(),
+            preps = [_oracle_prepare(li) for li in lis]
+            res = [_oracle_step(lis, preps, CPU_SAMPLE_ROWS) for _ in range(2)]
+            t, ops = min(res)
+            line["cpu_baseline"] = {"value": ops / t / 1e12, "unit": "TOPS", "cores": _cpu_threads(),
                                     "kind": "oracle",
-                                    "sample": f"{rows} of {M} rows (quantise + lora-down + fp64 forward), weights prepared untimed"}
+                                    "sample": f"{min(CPU_SAMPLE_ROWS, layers[0]['M'])} rows of each linear "
+                                              "(quantise + lora-down + fp64 forward), weights prepared untimed"}
         print(json.dumps(line), flush=True)
 
 
@@ -398,10 +481,8 @@ def run_stack(args, rank, world, local_rank):
         step()
     torch.cuda.synchronize()
     assert all(svdq.svdq_device_status(w) == 0 for (w, _, _, _, _) in layers)
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler = _sampler(local_rank)
     sampler.start()
-    time.sleep(0.1)
     _barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -450,10 +531,10 @@ def run_awq(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     svdq.load_library()
     stream = torch.cuda.current_stream()
-    li = synth.make_layer("awq", SEED, M=args.batch)
+    li = synth.make_layer("awq", 2, M=args.batch)
     M, K, N = li.shape.M, li.shape.K, li.shape.N
     W = torch.from_numpy(li.w).to(dev)
-    alpha = torch.from_numpy(synth.awq_alpha(K, SEED)).to(dev)
+    alpha = torch.from_numpy(synth.awq_alpha(K, 2)).to(dev)
     b = torch.from_numpy(li.bias_bits.view(np.int16)).to(dev)
     w = svdq.prepare_layer(W, alpha, None, None, b, 0, svdq.SVDQ_AWQ_W4A16)
     del W
@@ -464,10 +545,8 @@ def run_awq(args, rank, world, local_rank):
         flush.sum()
         svdq.svdq_awq_w4a16_forward(w, X, M, Y, svdq.SVDQ_OUT_BF16, stream)
     torch.cuda.synchronize()
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                           else os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank])
+    sampler = _sampler(local_rank)
     sampler.start()
-    time.sleep(0.1)
     _barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -531,9 +610,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rows", type=int, default=None, help="override M (smaller profiling cases only)")
-    ap.add_argument("--workload", default="qkv", choices=["qkv", "stack", "awq"],
-                    help="qkv: the single-layer bench line; stack: one denoising step of the block stack; "
-                         "awq: the awq_w4a16 modulation projection")
+    ap.add_argument("--workload", default="mlp", choices=["mlp", "qkv", "int4", "tiny", "stack", "awq"],
+                    help="mlp (default): the FLUX MLP pair; qkv: the fused QKV projection; int4: the INT4 "
+                         "batch of four images; tiny: the 64-row case; stack: one denoising step of the block "
+                         "stack; awq: the awq_w4a16 modulation projection")
     ap.add_argument("--batch", type=int, default=1, help="rows of the awq workload (images)")
     ap.add_argument("--blocks", type=int, default=57, help="blocks of the stack workload")
     ap.add_argument("--scale", default="static", choices=["static", "dynamic", "chain"],
@@ -546,11 +626,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    import synth
     if args.impl == "reference":
-        if rank == 0:
-            li = synth.make_layer(WORKLOAD, SEED)
-            run_reference(args, li, rank, world)
+        if args.workload not in LAYER_WORKLOADS:
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": f"the oracle arm covers the single-layer "
+                                  f"workloads {sorted(LAYER_WORKLOADS)}, not {args.workload}"}), flush=True)
+            return
+        run_reference(args, rank, world)
         return
     if world > 1:
         import datetime
@@ -558,17 +640,13 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    if args.workload in ("stack", "awq"):
-        try:
-            (run_stack if args.workload == "stack" else run_awq)(args, rank, world, local_rank)
-        finally:
-            if world > 1:
-                import torch.distributed as dist
-                dist.destroy_process_group()
-        return
-    li = synth.make_layer(WORKLOAD, SEED, **({"M": args.rows} if args.rows else {}))
     try:
-        run_ours(args, li, rank, world, local_rank)
+        if args.workload == "stack":
+            run_stack(args, rank, world, local_rank)
+        elif args.workload == "awq":
+            run_awq(args, rank, world, local_rank)
+        else:
+            run_layers(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

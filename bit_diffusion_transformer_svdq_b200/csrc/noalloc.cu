@@ -48,14 +48,18 @@ svdq_status scratch_address(int dev, void** out) {
 extern "C" svdq_status svdq_linear_forward_noalloc(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
                                                    void* Y, int32_t out_dtype, void* stream) {
   using namespace svdq;
-  if (!w) return SVDQ_ERR_INVALID_ARG;
+  // the same argument errors as svdq_linear_forward, before the size check
+  if (!w || w->desc.precision == SVDQ_AWQ_W4A16) return SVDQ_ERR_INVALID_ARG;
   if (M < 0) return SVDQ_ERR_SHAPE;
   if (M == 0) return SVDQ_OK;
-  const size_t need = svdq_workspace_bytes(w, M);
-  if (need == 0 || need + 1024 > kNoAllocScratchBytes) return SVDQ_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDev) return SVDQ_ERR_INVALID_ARG;
+  // the scratch used is the current device's copy of the array: the weights
+  // must live on that device too
+  if (w->device != dev) return SVDQ_ERR_INVALID_ARG;
+  const size_t need = svdq_workspace_bytes(w, M);
+  if (need == 0 || need + 1024 > kNoAllocScratchBytes) return SVDQ_ERR_WORKSPACE;
   svdq_status st = svdq_check_device(dev);
   if (st != SVDQ_OK) return st;
   void* base = nullptr;

@@ -54,6 +54,11 @@ class WeightsView(ctypes.Structure):
                 ("inv_lambda", ctypes.c_void_p), ("bias", ctypes.c_void_p)]
 
 
+class WeightsExport(ctypes.Structure):
+    _fields_ = [("qw", ctypes.c_void_p), ("sw", ctypes.c_void_p), ("l1s", ctypes.c_void_p), ("l2", ctypes.c_void_p),
+                ("inv_lambda", ctypes.c_void_p), ("bias", ctypes.c_void_p), ("g_w", ctypes.c_void_p)]
+
+
 class QkvPrologue(ctypes.Structure):
     """svdq_qkv_prologue: the attention prologue of a fused QKV projection
     (per-head RMS normalisation of Q and K with weights norm_q / norm_k,
@@ -93,6 +98,8 @@ _SIGS = {
     "svdq_prepare_weights": (_I, [ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P, _Z, ctypes.POINTER(_P), _P]),
     "svdq_weights_destroy": (None, [_P]),
     "svdq_weights_get_view": (_I, [_P, ctypes.POINTER(WeightsView)]),
+    "svdq_export_weights": (_I, [_P, ctypes.POINTER(WeightsExport), _P]),
+    "svdq_export_act_scales": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_global_scale": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_amax": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_scale_bytes": (_Z, [_P, _I]),
@@ -210,6 +217,35 @@ def svdq_prepare_weights(desc: LayerDesc, W, lam, L1, L2, bias, storage: torch.T
                                                _ptr(storage), storage.numel() * storage.element_size(),
                                                ctypes.byref(out), _stream(stream)), "svdq_prepare_weights")
     return Weights(out.value, storage, desc)
+
+
+def svdq_export_weights(w: Weights, stream=None) -> dict:
+    """Canonical host copies of prepared weights (numpy arrays): qw (N x K/2
+    packed codes), sw (N x K/16 E4M3 bytes, or N x K/64 float16), l1s
+    (rank x K bf16 bits), l2 (N x rank fp32), inv_lambda (K), bias (N), g_w."""
+    import numpy as np
+    v = w.view()
+    K, N, r = v.K, v.N, v.rank
+    out = dict(qw=np.empty((N, K // 2), np.uint8),
+               sw=np.empty((N, K // 16), np.uint8) if v.precision == SVDQ_NVFP4 else np.empty((N, K // 64), np.float16),
+               l1s=np.empty((r, K), np.uint16), l2=np.empty((N, r), np.float32),
+               inv_lambda=np.empty(K, np.float32), bias=np.empty(N, np.float32), g_w=np.empty(1, np.float32))
+    ex = WeightsExport(*(out[k].ctypes.data if out[k].size else None
+                         for k in ("qw", "sw", "l1s", "l2", "inv_lambda", "bias", "g_w")))
+    _check(load_library().svdq_export_weights(w.handle, ctypes.byref(ex), _stream(stream)), "svdq_export_weights")
+    out["g_w"] = np.float32(out["g_w"][0])
+    return out
+
+
+def svdq_export_act_scales(w: Weights, sx, M: int, stream=None):
+    """Canonical host copy of activation scales: M x K/16 E4M3 bytes (NVFP4)
+    or M x K/64 float16 (INT4)."""
+    import numpy as np
+    v = w.view()
+    out = np.empty((M, v.K // 16), np.uint8) if v.precision == SVDQ_NVFP4 else np.empty((M, v.K // 64), np.float16)
+    _check(load_library().svdq_export_act_scales(w.handle, _ptr(sx), M, out.ctypes.data if out.size else None,
+                                                 _stream(stream)), "svdq_export_act_scales")
+    return out
 
 
 def svdq_act_global_scale(w: Weights, X: torch.Tensor, g_x: torch.Tensor, stream=None) -> None:

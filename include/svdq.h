@@ -190,6 +190,47 @@ SVDQ_API void svdq_weights_destroy(svdq_weights* w);
 
 SVDQ_API svdq_status svdq_weights_get_view(const svdq_weights* w, svdq_weights_view* view);
 
+/* Host buffers that svdq_export_weights fills, in the canonical row-major
+ * layouts of the pages' quantised layer (the svdq_w4a4 block of
+ * quantization_config, "Native Ladefunktion": 4-bit codes, group scales,
+ * the 16-bit low-rank pair, the smoothing factor and the bias).  Every
+ * pointer is [host], caller-owned, and may be NULL to skip that part.
+ *   qw          N x K/2 bytes, two codes per byte, even k in the low nibble
+ *               (NVFP4: E2M1 nibbles; INT4 and AWQ_W4A16: two's complement)
+ *   sw          NVFP4: N x K/16 E4M3 bytes; INT4, AWQ_W4A16: N x K/64 fp16
+ *   l1s         rank x K bf16 bit patterns: bf16(RN32(L1 * inv_lambda))
+ *   l2          N x rank fp32 (the bf16 values of L2, exact)
+ *   inv_lambda  K fp32
+ *   bias        N fp32 (bf16 values; zeros when no bias was given)
+ *   g_w         one fp32: the NVFP4 weight tensor scale (1 otherwise) */
+typedef struct svdq_weights_export {
+  uint8_t* qw;
+  void* sw;
+  uint16_t* l1s;
+  float* l2;
+  float* inv_lambda;
+  float* bias;
+  float* g_w;
+} svdq_weights_export;
+
+/* Copies prepared weights to the host buffers of `out`, untiling the
+ * kernels' layouts (svdq_weights_view) into the canonical ones above.
+ * SYNCHRONOUS: the copies run on `stream`, which is synchronised before
+ * the call returns.  Allocates host memory only (temporary staging).
+ * Errors: SVDQ_ERR_INVALID_ARG for a NULL handle or `out`, SVDQ_ERR_CUDA
+ * when a copy or the synchronisation fails. */
+SVDQ_API svdq_status svdq_export_weights(const svdq_weights* w, svdq_weights_export* out, void* stream);
+
+/* Canonical host copy of an activation scale buffer written by
+ * svdq_quantize_act_lora_down for M rows of weights `w`: NVFP4 -> M x K/16
+ * E4M3 bytes, INT4 -> M x K/64 fp16, both row-major (the tiled and the
+ * group-major device layouts are described with svdq_weights_view and
+ * svdq_act_scale_bytes).  sx [device], out [host].  SYNCHRONOUS on
+ * `stream`.  SVDQ_ERR_INVALID_ARG for AWQ_W4A16 weights (no activation
+ * quantisation there) or NULL buffers; M == 0 is a no-op. */
+SVDQ_API svdq_status svdq_export_act_scales(const svdq_weights* w, const void* sx, int32_t M, void* out,
+                                            void* stream);
+
 /* Static activation tensor scale for NVFP4: g_x = RN32(amax |X_hat| / 2688)
  * with X_hat = RN32(X * inv_lambda) (1 when amax is 0), written to
  * g_x [device] (one fp32).  X [device] M x K bf16, M >= 1. */
@@ -366,7 +407,10 @@ SVDQ_API svdq_status svdq_linear_forward_dyn(const svdq_weights* w, const uint16
  * fits; M = 9216 does not).  Allocates nothing: no cudaMalloc, cudaFree
  * or allocating library call.  The first call on each device looks up the
  * array's device address (with that device current), so make that first
- * call before any stream capture.  All calls on a device share the array
+ * call before any stream capture.  `w` must have been prepared on the
+ * current device, whose copy of the array the call uses (another device's
+ * weights give SVDQ_ERR_INVALID_ARG, as do awq_w4a16 weights, before any
+ * size check).  All calls on a device share the array
  * and leave the last call's intermediates in it; every call rewrites all
  * it reads, so nothing needs clearing, but calls that overlap on the GPU
  * (other streams, other host threads) race on it. */

@@ -9,6 +9,7 @@ import numpy as np
 import torch
 
 import synth
+from oracle import formats as F
 from oracle import svdq as V
 
 PREC = {"nvfp4": 0, "int4": 1}
@@ -130,3 +131,122 @@ def y_error_stats(y: np.ndarray, ref: np.ndarray) -> dict:
     d = y.astype(np.float64) - ref
     rms = float(np.sqrt(np.mean(ref ** 2)))
     return dict(rel_f=float(np.linalg.norm(d) / np.linalg.norm(ref)), max_abs_over_rms=float(np.abs(d).max() / rms))
+
+
+def expected_weights(li: synth.LayerInputs, prep: V.Prepared) -> dict:
+    """The oracle's prepared weights in the canonical layout that
+    svdq_export_weights writes (codes packed two per byte, even k low)."""
+    qw = prep.qw if prep.precision == "nvfp4" else F.int4_to_nibble(prep.qw)
+    sw = prep.sw if prep.precision == "nvfp4" else prep.sw.view(np.uint16)
+    return dict(precision=prep.precision, g_w=np.float32(prep.g_w), inv_lambda=prep.inv_lam,
+                qw=F.pack_nibbles(qw), sw=sw, l1s=bf16_bits(prep.L1s).reshape(prep.rank, -1),
+                l2=prep.L2.reshape(-1, prep.rank), bias=li.bias)
+
+
+def check_weights_exact(svdq, w, exp: dict) -> None:
+    """Every prepared-weight part, exported in canonical layout through the C
+    ABI (svdq_export_weights), bit-exact against the oracle's preparation
+    (`exp` from expected_weights)."""
+    e = svdq.svdq_export_weights(w)
+    assert e["g_w"] == exp["g_w"]
+    assert np.array_equal(e["inv_lambda"].view(np.uint32), exp["inv_lambda"].view(np.uint32))
+    assert np.array_equal(e["qw"], exp["qw"])
+    sw = e["sw"] if exp["precision"] == "nvfp4" else e["sw"].view(np.uint16)
+    assert np.array_equal(sw, exp["sw"])
+    assert np.array_equal(e["l1s"], exp["l1s"])
+    assert np.array_equal(e["l2"], exp["l2"])
+    assert np.array_equal(e["bias"], exp["bias"])
+
+
+def lora_scale(ol: OracleLayer, precision: str) -> np.float32:
+    """The unit the kernels store lora_act in: RN32(1 / RN32(g_x g_w)) for
+    NVFP4, 1 for INT4."""
+    if precision != "nvfp4":
+        return np.float32(1.0)
+    return np.float32(1.0) / np.float32(np.float32(ol.gx) * ol.prep.g_w)
+
+
+def expected_act(x: np.ndarray, prep: V.Prepared, gx) -> dict:
+    """The oracle's activation codes (packed), canonical scales and
+    lora_act (fp64, unscaled) for every row of x."""
+    act = V.quantize_activations(x, prep, gx)
+    qx = act.qx if prep.precision == "nvfp4" else F.int4_to_nibble(act.qx)
+    sx = act.sx if prep.precision == "nvfp4" else act.sx.view(np.uint16)
+    return dict(precision=prep.precision, qx=F.pack_nibbles(qx), sx=sx, lora_act=act.lora_act, act=act)
+
+
+def check_act_exact(svdq, w, x: np.ndarray, ol: OracleLayer, qx, sx, la, exp: dict | None = None) -> dict:
+    """Activation codes and scales of every row bit-exact against the
+    oracle's quantiser (scales exported in canonical layout through the C
+    ABI, svdq_export_act_scales; padded scale rows zero), and lora_act
+    within the bound of the kernels' tf32 rounding."""
+    M, K = x.shape
+    if exp is None:
+        exp = expected_act(x, ol.prep, ol.gx)
+    precision = exp["precision"]
+    assert np.array_equal(qx[:M * K // 2].cpu().numpy().reshape(M, K // 2), exp["qx"])
+    sc = svdq.svdq_export_act_scales(w, sx, M)
+    assert np.array_equal(sc if precision == "nvfp4" else sc.view(np.uint16), exp["sx"])
+    mp = (M + 127) // 128 * 128
+    raw = sx.cpu().numpy()
+    if precision == "nvfp4":
+        assert np.all(raw[tiled_scale_index(mp, K)[M:]] == 0)
+    else:
+        assert np.all(raw[:mp * (K // 64) * 2].view(np.float16).reshape(K // 64, mp)[:, M:] == 0)
+    if la is not None:
+        r = ol.prep.rank
+        scale = float(lora_scale(ol, precision))
+        ref = exp["lora_act"] * scale
+        got = la[:M].cpu().numpy()
+        mag = exp.get("lora_mag")
+        if mag is None:
+            mag = np.abs(x).astype(np.float64) @ np.abs(ol.prep.L1s).astype(np.float64).T
+        mag = mag * scale
+        assert np.all(np.abs(got[:, :r].astype(np.float64) - ref) <= 2.0 ** -11 * np.abs(ref) + 1e-5 * mag + 1e-30)
+        assert np.all(got[:, r:] == 0)
+    return exp
+
+
+def check_y(y: np.ndarray, ref: np.ndarray, out_dtype: int, rel_f: float = 2e-3, max_abs: float = 1e-2,
+            widen: float = 1.0, ref_for_scale: np.ndarray | None = None) -> None:
+    """The output bar: relative Frobenius error <= rel_f; fp32 output
+    (out_dtype 1): max |error| <= max_abs rms(Y*); bf16 output: per element
+    |error| <= max_abs rms(Y*) + half a bf16 ulp of Y*.  `widen` scales both
+    bounds (a Lipschitz activation after the layer); `ref_for_scale` is the
+    pre-activation Y* whose norm and rms set them."""
+    base = ref if ref_for_scale is None else ref_for_scale
+    d = y.astype(np.float64) - ref
+    assert np.linalg.norm(d) <= widen * rel_f * np.linalg.norm(base)
+    rms = np.sqrt(np.mean(base ** 2))
+    if out_dtype:
+        assert np.abs(d).max() <= widen * max_abs * rms
+    else:
+        half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
+        assert np.all(np.abs(d) <= widen * max_abs * rms + half_ulp)
+
+
+def stack_linear_expected(args) -> dict:
+    """Oracle side of one linear of the denoising stack (block `blk`, layer
+    `j`), for a spawn worker: the layer inputs, the oracle's smoothing
+    factor and low-rank factors (inputs of the GPU preparation too), its
+    prepared weights and activation codes in canonical layout, and the fp64
+    Y* of `n_rows` seeded sampled rows."""
+    blk, j, n_rows, threads = args
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(threads):
+        name = synth.STACK_LAYERS[j]
+        li = synth.make_layer(name, synth.stack_seed(blk, j))
+        ol = oracle_layer(li)
+        ew = expected_weights(li, ol.prep)
+        ea = expected_act(li.x, ol.prep, ol.gx)
+        # the magnitude that bounds the lora_act rounding (see check_act_exact)
+        ea["lora_mag"] = np.abs(li.x).astype(np.float64) @ np.abs(ol.prep.L1s).astype(np.float64).T
+        M = li.shape.M
+        rows = np.sort(np.random.default_rng(1000 + 4 * blk + j).choice(M, n_rows, replace=False))
+        act = ea.pop("act")
+        sub = V.ActQuant(act.qx[rows], act.sx[rows], act.lora_act[rows])
+        ref = V.forward_from_codes(sub, ol.prep, ol.gx)
+    ol.prep.R = None  # not needed past the preparation; keeps the transfer small
+    ol.prep.qw = None
+    return dict(blk=blk, j=j, name=name, x_bits=li.x_bits, w=li.w, bias_bits=li.bias_bits, bias=li.bias,
+                ol=ol, exp_w=ew, exp_a=ea, rows=rows, ref=ref)

@@ -1,7 +1,8 @@
 """Parity at the full workload sizes, in the launch configuration the bench
-uses: every weight and activation code and scale bit-exact against the
-oracle; Y checked on seeded sampled rows (rows are independent given the
-codes, so the oracle computes only those rows)."""
+uses: every weight part and every activation code and scale of every row
+bit-exact against the oracle (weights and scales exported in canonical
+layout through the C ABI); Y checked on seeded sampled rows (rows are
+independent given the codes, so the oracle computes only those rows)."""
 import numpy as np
 import pytest
 import torch
@@ -26,111 +27,33 @@ def svdq():
     return mod
 
 
-@pytest.mark.parametrize("workload", ["qkv", "mlp_up", "mlp_down"])
-def test_full_size_nvfp4(svdq, workload):
-    li = synth.make_layer(workload, 2)
+def _rows_of(act: V.ActQuant, rows) -> V.ActQuant:
+    return V.ActQuant(act.qx[rows], act.sx[rows], act.lora_act[rows])
+
+
+@pytest.mark.parametrize("workload,seed,precision", [("qkv", 2, "nvfp4"), ("mlp_up", 2, "nvfp4"),
+                                                     ("mlp_down", 3, "nvfp4"), ("int4", 4, "int4")])
+def test_full_size(svdq, workload, seed, precision):
+    """The FLUX fused QKV projection, both MLP linears and the INT4 batch of
+    four images: all weight parts and all activation codes and scales
+    bit-exact; Y on sampled rows in both output types."""
+    li = synth.make_layer(workload, seed)
     M, K, N = li.shape.M, li.shape.K, li.shape.N
-    ol = T.oracle_layer(li)
-    w = T.gpu_prepare(svdq, li, ol)
-    h = T.weights_to_host(w)
-    assert h["g_w"] == ol.prep.g_w
-    assert np.array_equal(T.unpack_codes(h["qw"]), ol.prep.qw)
-    assert np.array_equal(T.untile_nvfp4_scales(h["sw"], N, K), ol.prep.sw)
+    ol = T.oracle_layer(li, precision=precision)
+    w = T.gpu_prepare(svdq, li, ol, precision)
+    T.check_weights_exact(svdq, w, T.expected_weights(li, ol.prep))
 
     X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
+    exp = T.check_act_exact(svdq, w, li.x, ol, qx, sx, la)
     rows = np.sort(np.random.default_rng(7).choice(M, SAMPLE_ROWS, replace=False))
-    xs = li.x[rows]
-    act = V.quantize_activations(xs, ol.prep, ol.gx)
-    codes = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
-    assert np.array_equal(codes[rows], act.qx)
-    assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K)[rows], act.sx)
-
-    ref = V.forward_from_codes(act, ol.prep, ol.gx)
-    rms = np.sqrt(np.mean(ref ** 2))
+    ref = V.forward_from_codes(_rows_of(exp["act"], rows), ol.prep, ol.gx if precision == "nvfp4" else None)
     for out_dtype in (1, 0):
         Y = torch.empty((M, N), dtype=torch.float32 if out_dtype else torch.bfloat16, device="cuda")
         svdq.svdq_w4a4_gemm_lora_up(w, qx, sx, float(ol.gx), la, M, Y, out_dtype)
         torch.cuda.synchronize()
-        y = Y.float().cpu().numpy()[rows].astype(np.float64)
-        d = y - ref
-        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F
-        if out_dtype:
-            assert np.abs(d).max() <= MAX_ABS * rms
-        else:
-            half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
-            assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
-        assert np.all(np.isfinite(Y.float().cpu().numpy()))
+        T.check_y(Y[torch.from_numpy(rows).cuda()].float().cpu().numpy(), ref, out_dtype, REL_F, MAX_ABS)
+        assert bool(torch.isfinite(Y.float()).all())
     assert svdq.svdq_device_status(w) == 0
-
-
-def test_full_size_int4(svdq):
-    """The INT4 configuration (four images: 18432 x 3072 -> 3072, rank 32)
-    at full size: every CTA of the persistent INT4 GEMM runs many tiles."""
-    li = synth.make_layer("int4", 4)
-    M, K, N = li.shape.M, li.shape.K, li.shape.N
-    ol = T.oracle_layer(li, precision="int4")
-    w = T.gpu_prepare(svdq, li, ol, "int4")
-    h = T.weights_to_host(w)
-    assert np.array_equal(T.unpack_codes(h["qw"]), (ol.prep.qw.astype(np.int16) & 0xF).astype(np.uint8))
-    sw = h["sw"].view(np.float16).reshape(K // 64, h["n_pad"])[:, :N].T
-    assert np.array_equal(sw.view(np.uint16), ol.prep.sw.view(np.uint16))
-
-    X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, 1.0)
-    rows = np.sort(np.random.default_rng(8).choice(M, SAMPLE_ROWS, replace=False))
-    act = V.quantize_activations(li.x[rows], ol.prep)
-    codes = T.nibbles_to_int(T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2)))
-    assert np.array_equal(codes[rows], act.qx)
-    mp = (M + 127) // 128 * 128
-    sxh = sx.cpu().numpy().view(np.float16).reshape(K // 64, mp)
-    assert np.array_equal(sxh[:, rows].T.view(np.uint16), act.sx.view(np.uint16))
-
-    ref = V.forward_from_codes(act, ol.prep)
-    rms = np.sqrt(np.mean(ref ** 2))
-    for out_dtype in (1, 0):
-        Y = torch.empty((M, N), dtype=torch.float32 if out_dtype else torch.bfloat16, device="cuda")
-        svdq.svdq_w4a4_gemm_lora_up(w, qx, sx, 1.0, la, M, Y, out_dtype)
-        torch.cuda.synchronize()
-        y = Y.float().cpu().numpy()[rows].astype(np.float64)
-        d = y - ref
-        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F
-        if out_dtype:
-            assert np.abs(d).max() <= MAX_ABS * rms
-        else:
-            half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
-            assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
-        assert np.all(np.isfinite(Y.float().cpu().numpy()))
-    assert svdq.svdq_device_status(w) == 0
-
-
-def test_stack_block_through_forward(svdq):
-    """One block of the 57-block denoising stack at full size (QKV 3072 ->
-    9216, out 3072 -> 3072, MLP up 3072 -> 12288, down 12288 -> 3072; M =
-    4608, rank 32, NVFP4), every linear through svdq_linear_forward with the
-    per-layer seeds of the stack: sampled codes and scales bit-exact, sampled
-    Y rows within the bf16-output tolerance."""
-    for layer, name in enumerate(synth.STACK_LAYERS):
-        li = synth.make_layer(name, synth.stack_seed(0, layer))
-        M, K, N = li.shape.M, li.shape.K, li.shape.N
-        ol = T.oracle_layer(li)
-        w = T.gpu_prepare(svdq, li, ol)
-        rows = np.sort(np.random.default_rng(100 + layer).choice(M, 64, replace=False))
-        act = V.quantize_activations(li.x[rows], ol.prep, ol.gx)
-        X, qx, sx, la = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
-        codes = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
-        assert np.array_equal(codes[rows], act.qx), name
-        assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K)[rows], act.sx), name
-        ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
-        Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-        svdq.svdq_linear_forward(w, X, M, float(ol.gx), Y, ws, ws.numel(), 0)
-        torch.cuda.synchronize()
-        assert svdq.svdq_device_status(w) == 0
-        ref = V.forward_from_codes(act, ol.prep, ol.gx)
-        y = Y.float().cpu().numpy()[rows].astype(np.float64)
-        d = y - ref
-        rms = np.sqrt(np.mean(ref ** 2))
-        assert np.linalg.norm(d) / np.linalg.norm(ref) <= REL_F, name
-        half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
-        assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp), name
 
 
 def test_full_size_qkv_prologue(svdq):
@@ -158,15 +81,7 @@ def test_full_size_qkv_prologue(svdq):
         torch.cuda.synchronize()
         y = Y.float().cpu().numpy()[rows].astype(np.float64)
         for sec in range(3):
-            r_ = ref[:, sec * wd:(sec + 1) * wd]
-            d = y[:, sec * wd:(sec + 1) * wd] - r_
-            rms = np.sqrt(np.mean(r_ ** 2))
-            assert np.linalg.norm(d) / np.linalg.norm(r_) <= REL_F
-            if out_dtype:
-                assert np.abs(d).max() <= MAX_ABS * rms
-            else:
-                half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(r_), 1e-30))) - 8)
-                assert np.all(np.abs(d) <= MAX_ABS * rms + half_ulp)
+            T.check_y(y[:, sec * wd:(sec + 1) * wd], ref[:, sec * wd:(sec + 1) * wd], out_dtype, REL_F, MAX_ABS)
     assert svdq.svdq_device_status(w) == 0
 
 
@@ -198,12 +113,7 @@ def test_full_size_mlp_chain(svdq):
     act = V.quantize_activations(li_a.x[rows], ol_a.prep, ol_a.gx)  # ol_a.gx: the dynamic scale of all of X
     ystar = V.forward_from_codes(act, ol_a.prep, ol_a.gx)
     ref = C.gelu_tanh(ystar)
-    y = Ya.float().cpu().numpy()[rows].astype(np.float64)
-    d = y - ref
-    rms = np.sqrt(np.mean(ystar ** 2))
-    assert np.linalg.norm(d) <= 1.13 * REL_F * np.linalg.norm(ystar)
-    half_ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 8)
-    assert np.all(np.abs(d) <= 1.13 * MAX_ABS * rms + half_ulp)
+    T.check_y(Ya.float().cpu().numpy()[rows], ref, 0, REL_F, MAX_ABS, widen=1.13, ref_for_scale=ystar)
     a2 = torch.empty(1, dtype=torch.float32, device="cuda")
     svdq.svdq_act_amax(wb, Ya.view(torch.int16), a2)
     amax = np.float32(words[1].item())

@@ -18,10 +18,6 @@ from tests import svdq_testlib as T
 
 pytestmark = pytest.mark.gpu
 
-REL_F = 2e-3
-MAX_ABS = 1e-2
-
-
 @pytest.fixture(scope="module")
 def svdq():
     if not torch.cuda.is_available():
@@ -31,28 +27,33 @@ def svdq():
     return mod
 
 
-def _close(y, ref):
-    d = y.astype(np.float64) - ref.astype(np.float64)
-    rms = np.sqrt(np.mean(ref.astype(np.float64) ** 2))
-    rel_f = np.linalg.norm(d) / np.linalg.norm(ref.astype(np.float64))
-    assert rel_f <= REL_F and np.abs(d).max() <= MAX_ABS * rms, (rel_f, np.abs(d).max() / rms)
-
-
 def test_noalloc_forward_matches_workspace_forward_twice(svdq):
-    li = synth.make_layer("qkv", 31, M=333, K=1024, N=768)
+    """Two calls in a row, the second with fewer rows than the first, so that
+    it runs over the first call's leftovers in the shared scratch: each must
+    equal the workspace forward bit for bit (same kernels, same inputs), and
+    the second call must leave device memory use unchanged."""
+    K, N = 1024, 768
+    li = synth.make_layer("qkv", 31, M=333, K=K, N=N)
     ol = T.oracle_layer(li)
     w = T.gpu_prepare(svdq, li, ol)
-    M, N = li.shape.M, li.shape.N
-    ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
-    x2 = synth.make_layer("qkv", 32, M=M, K=1024, N=768).x_bits
-    for x_bits in (li.x_bits, x2):
+    x2 = synth.make_layer("qkv", 32, M=200, K=K, N=N).x_bits
+    for call, x_bits in enumerate((li.x_bits, x2)):
+        M = x_bits.shape[0]
+        ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
         X = T.dev_u16(x_bits)
-        ref = torch.empty((M, N), dtype=torch.float32, device="cuda")
-        svdq.svdq_linear_forward(w, X, M, float(ol.gx), ref, ws, ws.numel(), svdq.SVDQ_OUT_F32)
-        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
-        svdq.svdq_linear_forward_noalloc(w, X, M, float(ol.gx), y, svdq.SVDQ_OUT_F32)
-        torch.cuda.synchronize()
-        _close(y.cpu().numpy(), ref.cpu().numpy())
+        for out_dtype, dt in ((svdq.SVDQ_OUT_F32, torch.float32), (svdq.SVDQ_OUT_BF16, torch.bfloat16)):
+            ref = torch.empty((M, N), dtype=dt, device="cuda")
+            svdq.svdq_linear_forward(w, X, M, float(ol.gx), ref, ws, ws.numel(), out_dtype)
+            y = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+            torch.cuda.synchronize()
+            if call == 1:
+                alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+            svdq.svdq_linear_forward_noalloc(w, X, M, float(ol.gx), y, out_dtype)
+            torch.cuda.synchronize()
+            if call == 1:
+                assert torch.cuda.memory_allocated() == alloc0
+                assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.equal(y, ref), (call, out_dtype)
     assert svdq.svdq_device_status(w) == 0
 
 
@@ -66,3 +67,18 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(svdq):
     with pytest.raises(svdq.SVDQError) as e:
         svdq.svdq_linear_forward_noalloc(w, X, M, float(ol.gx), Y)
     assert e.value.status == 7
+
+
+def test_noalloc_rejects_awq_weights_before_the_size_check(svdq):
+    """awq_w4a16 weights have no activation quantisation: an argument error,
+    whatever M, as in svdq_linear_forward."""
+    li = synth.make_layer("awq", 5, M=4, K=256, N=256)
+    W = T.dev_f32(li.w)
+    w = svdq.prepare_layer(W, torch.ones(256, dtype=torch.float32, device="cuda"), None, None, T.dev_u16(li.bias_bits),
+                           0, svdq.SVDQ_AWQ_W4A16)
+    M = 1 << 20
+    X = torch.zeros((16, 256), dtype=torch.int16, device="cuda")
+    Y = torch.empty((16, 256), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(svdq.SVDQError) as e:
+        svdq.svdq_linear_forward_noalloc(w, X, M, 1.0, Y)
+    assert e.value.status == 1
