@@ -110,7 +110,7 @@ bool encode_tmap_chunked_bf16(CUtensorMap* tm, const void* base, uint64_t rows, 
                               uint32_t box_chunks);
 
 // 64-column chunks per stage of the activation quantiser (the L1s map's box).
-constexpr int kQChunks = 4;
+constexpr int kQChunks = 1;
 
 int num_sms(int device);
 
