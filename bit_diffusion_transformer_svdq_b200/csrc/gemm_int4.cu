@@ -1,42 +1,44 @@
 // INT4 (group 64) variant of the 4-bit GEMM with the low-rank up-projection
 // fused in: Y = sum_g s_x[m,g] s_w[n,g] (sum_{k in g} qx qw) + lora_act L2^T + b.
-// The 4-bit codes are unpacked to 8 bits and multiplied with tcgen05
-// kind::i8 MMAs (int32 accumulate); the scales change with every 64-group,
-// so each group's integer product leaves TMEM and is scaled into an fp32
-// accumulator held in registers.
+// tcgen05 has no 4-bit integer kind, so the codes go to the tensor core as
+// 8-bit operands: E4M3 bytes, which hold every integer in [-8, 7] exactly,
+// multiplied by kind::f8f6f4 MMAs into fp32 TMEM accumulators.  Every
+// product is an integer of magnitude at most 64 and a group's sum at most
+// 4096, so the accumulator holds each group's integer dot product exactly,
+// as a float; the scales change with every 64-group, so each group's
+// product leaves TMEM and is scaled into an fp32 accumulator held in
+// registers: acc += RN(P s_w) s_x.
 //
 // sm_100a design, one CTA per 128 x 128 output tile (persistent over the
 // tile list):
 //   warp 0      TMA producer: per ring stage (128 K = two groups) the packed
 //               activation codes (128 rows x 64 B, 64-byte swizzled) and the
-//               prepared int8 weight codes (128 rows x 128 B, 128-byte
-//               swizzled); per tile one stage of lora_act / L2 (fp32).
-//   warps 2-3   converters: two rows per lane, unpack the packed activation
-//               codes into int8 in the 128-byte-swizzled layout of the MMA
-//               operand (same K permutation as the prepared weights).
-//   warp 1      TMEM owner and MMA issuer: per group two kind::i8 MMAs
-//               (K = 32) into one of four int32 accumulators (128 columns
+//               prepared E4M3 weight codes (128 rows x 128 B, 128-byte
+//               swizzled); per tile one stage of lora_act / L2 (fp32); per
+//               group the tile's 128 fp32 s_w and 128 fp16 s_x into a ring
+//               of eight shared-memory entries (released with one arrival per
+//               epilogue warp).
+//   warps 2-3   converters: two rows per lane, turn the packed codes into
+//               E4M3 bytes in the 128-byte-swizzled layout of the MMA operand
+//               (a byte permute through a 16-entry table, natural K order).
+//   warp 1      TMEM owner and MMA issuer: per group two kind::f8f6f4 MMAs
+//               (K = 32) into one of four fp32 accumulators (128 columns
 //               each), so the MMAs run up to three groups ahead of the
 //               scaling; per tile four kind::tf32 MMAs of the lora-up into
 //               the next accumulator, as one more "group" of scale 1.
 //   warps 4-19  epilogue: warp e = w - 4 owns rows 32 (e % 4) .. + 31 (its
 //               TMEM lane quarter) and columns 32 (e / 4) .. + 31; per group
-//               it reads its int32 products, frees the accumulator and adds
-//               RN(P s_w) s_x to its fp32 accumulator.  RN(P s_w) is one FMA
-//               on the bit pattern magic + P (exact for |P| < 2^22; a
-//               group's |P| is at most 64 * 8 * 8), no int-to-float
-//               conversion.  The producer bulk-copies each group's scales
-//               into a ring of eight shared-memory entries (released with
-//               one arrival per epilogue warp), so the 16 warps never wait
-//               for one another between groups.  Finally y = acc + b is
-//               stored; the QKV variant first applies the attention
-//               prologue (per 128-column head of Q and K: RMS
-//               normalisation, weight, rotary embedding), the four column
-//               slices of a row adding their sums of squares through shared
-//               memory.
-// The group rescale is CUDA-core work on every output element (three
-// operations per element per 64 K, against 64 MACs on the tensor core), so
-// this kernel is bound by it, not by the MMAs.
+//               it reads its products, frees the accumulator and adds
+//               RN(P s_w) s_x to its fp32 accumulator with packed two-wide
+//               multiplies and FMAs, the 32 column scales read as eight
+//               broadcast 16-byte loads.  Finally y = acc + b is stored; the
+//               QKV variant first applies the attention prologue (per
+//               128-column head of Q and K: RMS normalisation, weight, rotary
+//               embedding), the four column slices of a row adding their sums
+//               of squares through shared memory.
+// The group rescale is CUDA-core work on every output element (one packed
+// multiply and one packed FMA per two elements per 64 K, against 64 MACs on
+// the tensor core), so this kernel is bound by it, not by the MMAs.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -51,45 +53,55 @@ namespace {
 constexpr int kTileM = 128, kTileN = 128;
 constexpr int kI4Stages = 5;
 constexpr int kApBytes = kTileM * 64;    // packed activation codes of a stage: 128 K per row
-constexpr int kA8Bytes = kTileM * 128;   // unpacked
-constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes
+constexpr int kA8Bytes = kTileM * 128;   // the same codes as E4M3 bytes
+constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes (E4M3)
 constexpr int kI4StageBytes = kApBytes + kA8Bytes + kB8Bytes;  // 40 KB
-constexpr int kConvWarps = 2;  // each lane unpacks two rows (r, r + 64)
+constexpr int kConvWarps = 2;  // each lane converts two rows (r, r + 64)
 constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
 constexpr int kI4Threads = 32 * (2 + kConvWarps + kI4EpiWarps);
-constexpr int kAccBufs = 4;  // int32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
+constexpr int kAccBufs = 4;  // fp32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
 constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
 // Group scales reach the epilogue through a ring of kScaleSlots entries in
 // shared memory, filled by the producer with bulk copies: per entry the
-// tile's 128 (s_w, -magic s_w) pairs and its 128 fp16 s_x.
+// tile's 128 fp32 s_w and its 128 fp16 s_x.
 constexpr int kScaleSlots = 8;
-constexpr int kScaleSlotBytes = kTileN * 8 + kTileM * 2;  // 1280
+constexpr int kScaleSlotBytes = kTileN * 4 + kTileM * 2;  // 768
 constexpr int kScaleOff = kI4Stages * kI4StageBytes;
-// each epilogue warp's private copy of its current group's scales: 32
-// (s_w, -magic s_w) pairs and 32 s_x
-constexpr int kPrivOff = kScaleOff + kScaleSlots * kScaleSlotBytes;
-constexpr int kPrivBytes = 32 * 8 + 32 * 4;
-constexpr int kI4BarOff = kPrivOff + kI4EpiWarps * kPrivBytes;
+constexpr int kI4BarOff = kScaleOff + kScaleSlots * kScaleSlotBytes;
 constexpr int kI4RedOff = kI4BarOff + 512;  // QKV: one float per row and column slice (16 x 32)
 constexpr size_t kI4Smem = kI4RedOff + kI4EpiWarps * 32 * 4 + 1024 /*align*/;
 static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
 static_assert(kI4Smem <= 232448, "shared memory budget");
 
-// kind::i8: int32 D, signed 8-bit A and B, K-major, N = 128, M = 128.
-constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
+// kind::f8f6f4: fp32 D, E4M3 A and B, K-major, N = 128, M = 128.
+constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 // kind::tf32: fp32 D, tf32 A and B, K-major, N = 128, M = 128.
 constexpr uint32_t kIdescTf32x = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 
-// 64-byte-swizzle descriptor-free read of the packed codes: row r, 16-byte
-// unit j lives at r * 64 + ((j ^ ((r >> 1) & 3)) << 4).
-__device__ __forceinline__ uint32_t unpack_lo(uint32_t w) {
-  return (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
-__device__ __forceinline__ uint32_t unpack_hi(uint32_t w) { return unpack_lo(w >> 4); }
+
+// Eight packed two's-complement codes (element e in bits 4e .. 4e+3) to
+// eight E4M3 bytes in the same order.  A byte permute looks each nibble's
+// low three bits up in the tables of n = 0..7 and n = 8..15; a second
+// permute spreads each nibble's bit 3 to a byte mask (the top bit of byte j
+// of w is bit 3 of nibble 2j + 1, that of byte j of w << 4 bit 3 of nibble
+// 2j) that picks between the two.
+__device__ __forceinline__ uint2 e4m3x8(uint32_t w) {
+  const uint32_t w4 = w << 4;
+  const uint32_t s0 = w & 0x7777u, s1 = (w >> 16) & 0x7777u;
+  const uint32_t m0 = prmt(w4, w, 0xD9C8u), m1 = prmt(w4, w, 0xFBEAu);
+  const uint32_t lo0 = prmt(kI4E4m3Lo0, kI4E4m3Lo1, s0), hi0 = prmt(kI4E4m3Hi0, kI4E4m3Hi1, s0);
+  const uint32_t lo1 = prmt(kI4E4m3Lo0, kI4E4m3Lo1, s1), hi1 = prmt(kI4E4m3Hi0, kI4E4m3Hi1, s1);
+  return make_uint2((hi0 & m0) | (lo0 & ~m0), (hi1 & m1) | (lo1 & ~m1));
+}
 
 struct I4Params {
   const __half* sx;   // [K/64][m_pad]
-  const float2* swp;  // [K/64][n_pad / 2] x (s_w[2j], s_w[2j+1], -magic s_w[2j], -magic s_w[2j+1])
+  const float* sw32;  // [K/64][n_pad]
   const float* bias;
   void* Y;
   int* status;
@@ -103,6 +115,9 @@ struct I4Params {
   const float* rope_sin;
   float eps;
   int qk_cols;  // 2 * heads * 128; K starts at qk_cols / 2
+  // 0 at run time, unknown to the compiler: ANDing a loaded value with it
+  // gives a zero that still depends on the load (see the scale release)
+  uint32_t dep_mask;
 };
 
 template <bool kF32Out, bool kQkv>
@@ -208,8 +223,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
               const int g = 2 * kb + gi;
               uint8_t* dst = smem + kScaleOff + ss * kScaleSlotBytes;
               mbar_arrive_expect_tx(&sc_full[ss], kScaleSlotBytes);
-              bulk_load(dst, p.swp + static_cast<size_t>(g) * p.n_pad + n0, kTileN * 8, &sc_full[ss]);
-              bulk_load(dst + kTileN * 8, p.sx + static_cast<size_t>(g) * p.m_pad + m0, kTileM * 2, &sc_full[ss]);
+              bulk_load(dst, p.sw32 + static_cast<size_t>(g) * p.n_pad + n0, kTileN * 4, &sc_full[ss]);
+              bulk_load(dst + kTileN * 4, p.sx + static_cast<size_t>(g) * p.m_pad + m0, kTileM * 2, &sc_full[ss]);
             }
             __syncwarp();
             sc_mask |= 1u << ss;
@@ -229,6 +244,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
 #pragma unroll 1
           for (int rr = 0; rr < kTileM / (32 * kConvWarps); ++rr) {
             const int r = (rr * kConvWarps + warp - 2) * 32 + lane;  // row of the tile
+            // packed codes, 64-byte swizzled: row r's 16-byte unit j at r * 64 + ((j ^ ((r >> 1) & 3)) << 4)
             const uint8_t* ap = smem + stage * kI4StageBytes + r * 64;
             uint8_t* a8 = smem + stage * kI4StageBytes + kApBytes + r * 128;
             uint4 in[4];
@@ -237,9 +253,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             const uint32_t w[16] = {in[0].x, in[0].y, in[0].z, in[0].w, in[1].x, in[1].y, in[1].z, in[1].w,
                                     in[2].x, in[2].y, in[2].z, in[2].w, in[3].x, in[3].y, in[3].z, in[3].w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) =
-                  make_uint4(unpack_lo(w[2 * u]), unpack_hi(w[2 * u]), unpack_lo(w[2 * u + 1]), unpack_hi(w[2 * u + 1]));
+            for (int u = 0; u < 8; ++u) {  // 16 codes: k = 16 u .. 16 u + 15
+              const uint2 b0 = e4m3x8(w[2 * u]), b1 = e4m3x8(w[2 * u + 1]);
+              *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) = make_uint4(b0.x, b0.y, b1.x, b1.y);
+            }
           }
           fence_proxy_async_smem();
           __syncwarp();
@@ -270,8 +287,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           tc_fence_after();
           if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k)  // K = 32 int8 (32 bytes) per MMA
-              mma_i8(tmem + buf * kTileN, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescI8, k ? 1u : 0u);
+            for (int k = 0; k < 2; ++k)  // K = 32 E4M3 (32 bytes) per MMA
+              mma_f8(tmem + buf * kTileN, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescF8, k ? 1u : 0u);
             tc_commit(&acc_full[buf]);
           }
           __syncwarp();
@@ -305,18 +322,18 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   } else {
     // ---------------------------------------------------------- epilogue
     // warp e = 0..15 owns rows 32 (e % 4) .. + 31 (its TMEM lane quarter)
-    // and columns 32 (e / 4) .. + 31.  Per group it reads its 32 int32
-    // products, frees the accumulator (one arrival per warp) and adds
-    // RN(P s_w) s_x to its fp32 accumulator in registers.  The group's
-    // scales come from the producer's ring (waited for per warp, released
-    // with one arrival per warp): the warps never wait for one another.
+    // and columns 32 (e / 4) .. + 31.  Per group it reads its 32 products
+    // (fp32: exact integers), frees the accumulator (one arrival per warp)
+    // and adds RN(P s_w) s_x to its fp32 accumulator in registers.  The
+    // group's scales come from the producer's ring (waited for per warp,
+    // released with one arrival per warp): the warps never wait for one
+    // another.
     const int e = warp - 2 - kConvWarps;
     const int q4 = e & 3;
     const int cs = e >> 2;                  // column slice
     const int r = 32 * q4 + lane;           // row within the tile
     uint32_t gcount = 0;
     uint32_t sc_use = 0;  // scale-ring entries consumed
-    uint8_t* const priv = smem + kPrivOff + e * kPrivBytes;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
@@ -327,26 +344,10 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
       const int uses = groups + (p.n_lora > 0 ? 1 : 0);
       for (int g = 0; g < uses; ++g, ++gcount) {
-        float sxr = 0.0f;
-        // (s_w[c], s_w[c+1], -magic s_w[c], -magic s_w[c+1]) per float4:
-        // the two operand pairs of the packed FMA, broadcast reads of the
-        // warp's private copy
-        const float4* swq = reinterpret_cast<const float4*>(priv);
-        if (g < groups) {
-          // copy this warp's scales out of the ring entry, then release it:
-          // the stores consume the loaded values, so every load of the entry
-          // has completed before the arrival that lets the producer's next
-          // bulk copy overwrite it
-          const uint32_t ss = sc_use % kScaleSlots;
-          if (!mbar_wait(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) { ok = false; break; }
-          const uint8_t* sb = smem + kScaleOff + ss * kScaleSlotBytes;
-          reinterpret_cast<float2*>(priv)[lane] = reinterpret_cast<const float2*>(sb)[32 * cs + lane];
-          reinterpret_cast<float*>(priv + 256)[lane] =
-              __half2float(reinterpret_cast<const __half*>(sb + kTileN * 8)[r]);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sc_empty[ss]);
-          ++sc_use;
-          sxr = reinterpret_cast<const float*>(priv + 256)[lane];
+        const uint32_t ss = sc_use % kScaleSlots;  // this group's ring entry
+        if (g < groups && !mbar_wait(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) {
+          ok = false;
+          break;
         }
         const uint32_t buf = gcount % kAccBufs;
         if (!mbar_wait(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
@@ -358,20 +359,37 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the products are in registers: free the buffer
         if (g < groups) {
+          // the warp's 32 column scales, eight broadcast 16-byte loads; two
+          // columns per packed multiply (RN(P s_w)) and packed FMA (+ s_x)
+          const uint8_t* sb = smem + kScaleOff + ss * kScaleSlotBytes;
+          const float sxr = __half2float(reinterpret_cast<const __half*>(sb + kTileN * 4)[r]);
+          const float4* sw4 = reinterpret_cast<const float4*>(sb) + 8 * cs;
           const float2 sx2 = make_float2(sxr, sxr);
+          uint32_t dep = __float_as_uint(sxr);
 #pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float4 t = swq[c / 2];
-            // RN(P s_w) exactly: bits(magic) + P is the float magic + P; two
-            // columns per packed FMA
-            const float2 f = make_float2(__int_as_float(static_cast<int>(P[c]) + 0x4B400000),
-                                         __int_as_float(static_cast<int>(P[c + 1]) + 0x4B400000));
-            const float2 u = __ffma2_rn(f, make_float2(t.x, t.y), make_float2(t.z, t.w));
-            const float2 a = __ffma2_rn(u, sx2, make_float2(acc[c], acc[c + 1]));
-            acc[c] = a.x;
-            acc[c + 1] = a.y;
+          for (int q = 0; q < 8; ++q) {
+            const float4 t = ld_shared_f4_inorder(sw4 + q);
+            dep ^= __float_as_uint(t.x);
+            const float2 u0 = __fmul2_rn(make_float2(__uint_as_float(P[4 * q]), __uint_as_float(P[4 * q + 1])),
+                                         make_float2(t.x, t.y));
+            const float2 u1 = __fmul2_rn(make_float2(__uint_as_float(P[4 * q + 2]), __uint_as_float(P[4 * q + 3])),
+                                         make_float2(t.z, t.w));
+            const float2 a0 = __ffma2_rn(u0, sx2, make_float2(acc[4 * q], acc[4 * q + 1]));
+            const float2 a1 = __ffma2_rn(u1, sx2, make_float2(acc[4 * q + 2], acc[4 * q + 3]));
+            acc[4 * q] = a0.x;
+            acc[4 * q + 1] = a0.y;
+            acc[4 * q + 2] = a1.x;
+            acc[4 * q + 3] = a1.y;
           }
-          __syncwarp();  // the private copy is rewritten at the next group
+          // Release the ring entry.  The producer's next bulk copy may then
+          // overwrite it, so the arrival must follow the completion of every
+          // load of the entry above: its address depends on one value of
+          // each load, through a zero the compiler cannot fold away (a
+          // run-time mask that is 0).
+          const uint32_t zero = dep & p.dep_mask;
+          __syncwarp();
+          if (lane == 0) mbar_arrive_at(smem_u32(&sc_empty[ss]) + zero);
+          ++sc_use;
         } else {  // the lora-up, fp32
 #pragma unroll
           for (int c = 0; c < 32; ++c) acc[c] = __fadd_rn(acc[c], __uint_as_float(P[c]));
@@ -505,7 +523,7 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   }
   I4Params p;
   p.sx = static_cast<const __half*>(sx);
-  p.swp = w->swp;
+  p.sw32 = w->sw32;
   p.bias = w->bias;
   p.Y = Y;
   p.status = w->status;
@@ -521,6 +539,7 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   p.rope_sin = pro ? pro->rope_sin : nullptr;
   p.eps = pro ? pro->eps : 0.0f;
   p.qk_cols = pro ? 2 * pro->heads * pro->head_dim : 0;
+  p.dep_mask = 0;
   const int tiles = ((M + kTileM - 1) / kTileM) * ((N + kTileN - 1) / kTileN);
   const int grid = std::min(tiles, num_sms(w->device));
   const bool f32 = out_dtype == SVDQ_OUT_F32;

@@ -27,15 +27,18 @@ inline size_t int4_scale_bytes(int64_t rows_padded, int K) { return static_cast<
 struct WeightLayout {
   size_t qw, sw, l1s, l2, inv_lambda, bias, status, amax, total;
   size_t sw_bytes;
-  size_t qw8, swp;  // INT4 only (0 otherwise): unpacked int8 codes, float scale pairs
+  size_t qw8, sw32;  // INT4 only (0 otherwise): codes as E4M3 bytes, fp32 group scales
 };
 
-// INT4 working copies for the kind::i8 GEMM.  The tensor core takes 8-bit
-// operands, so the 4-bit codes are unpacked with one fixed permutation of K
-// inside every 8-value block: a packed word with nibbles k0..k7 becomes the
-// bytes k0 k2 k4 k6 k1 k3 k5 k7.  Both operands use it, so every dot
-// product (and every 64-group) is unchanged.
-constexpr float kI2FMagic = 12582912.0f;  // 1.5 * 2^23: bits(magic) + i = bits(magic + i), |i| < 2^22
+// INT4 working copies for the tensor-core GEMM.  tcgen05 has no 4-bit
+// integer kind, so the codes go to the tensor core as 8-bit operands: E4M3
+// bytes, which hold every integer in [-8, 7] exactly (kind::f8f6f4).  Each
+// product is an integer of magnitude at most 64 and a 64-group's sum at
+// most 4096, exact in the fp32 accumulator, so a group's TMEM result is the
+// integer dot product itself, already a float.  Codes keep their natural K
+// order.  E4M3 of the two's-complement nibble n: kI4E4m3[n].
+constexpr uint32_t kI4E4m3Lo0 = 0x44403800u, kI4E4m3Lo1 = 0x4E4C4A48u;  // n = 0..7: 0, 1, 2, ..., 7
+constexpr uint32_t kI4E4m3Hi0 = 0xCACCCED0u, kI4E4m3Hi1 = 0xB8C0C4C8u;  // n = 8..15: -8, -7, ..., -1
 WeightLayout weight_layout(const svdq_layer_desc& d);
 
 }  // namespace svdq
@@ -57,14 +60,14 @@ struct svdq_weights {
   int* status;    // written by the kernels when a bounded wait runs out
   uint32_t* amax; // scratch: [0], [1] the preparation's amax and g_w; [2], [3] the activation amax
                   // reduction (max, block count), zero between calls
-  int8_t* qw8;    // INT4: n_pad x K unpacked codes (K permuted as above); NVFP4: null
-  float2* swp;    // INT4: [K/64][n_pad / 2] x (s_w[2j], s_w[2j+1], -kI2FMagic s_w[2j], -kI2FMagic s_w[2j+1]); NVFP4: null
+  uint8_t* qw8;   // INT4: n_pad x K codes as E4M3 bytes (rows past N zero); NVFP4: null
+  float* sw32;    // INT4: [K/64][n_pad] group scales as fp32; NVFP4: null
   int device;
   CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_sw;  // NVFP4 weight scales viewed as rows of 256 bytes, boxes of 8 rows (4 atoms)
   CUtensorMap tm_l1s; // bf16 L1s as 64-column chunks: boxes of all rank_pad rows x kQChunks chunks
-  CUtensorMap tm_qw8; // INT4: unpacked codes, 128-byte swizzled boxes of 128 rows x 128 K
+  CUtensorMap tm_qw8; // INT4: E4M3 codes, 128-byte swizzled boxes of 128 rows x 128 K
 };
 
 namespace svdq {

@@ -147,12 +147,10 @@ __global__ void quantize_weights_kernel(const float* __restrict__ W, const float
   }
 }
 
-// INT4 working copies: unpacked codes (K permuted within 8-value blocks,
-// rows N..n_pad zero) and the float scales, per group and column pair
-// (s_w[2j], s_w[2j+1], -kI2FMagic s_w[2j], -kI2FMagic s_w[2j+1]): the two
-// operand pairs of the epilogue's packed FMA.
-__global__ void int4_unpack_kernel(const uint8_t* __restrict__ qw, const __half* __restrict__ sw, int N, int K,
-                                   int64_t n_pad, int8_t* __restrict__ qw8, float2* __restrict__ swp) {
+// INT4 working copies: the codes as E4M3 bytes in natural K order (rows
+// N..n_pad zero) and the group scales as fp32, [K/64][n_pad].
+__global__ void int4_e4m3_kernel(const uint8_t* __restrict__ qw, const __half* __restrict__ sw, int N, int K,
+                                 int64_t n_pad, uint8_t* __restrict__ qw8, float* __restrict__ sw32) {
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   const size_t blocks = static_cast<size_t>(n_pad) * (K / 8);
   if (i < blocks) {
@@ -161,20 +159,20 @@ __global__ void int4_unpack_kernel(const uint8_t* __restrict__ qw, const __half*
     uint2 out = make_uint2(0u, 0u);
     if (n < N) {
       const uint32_t w = *reinterpret_cast<const uint32_t*>(qw + static_cast<size_t>(n) * (K / 2) + 4 * j);
-      // nibble -> signed byte without carries between bytes: ((v ^ 8) + 0x78) ^ 0x80
-      out.x = (((w & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
-      out.y = ((((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u) + 0x78787878u) ^ 0x80808080u;
+      uint32_t b[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t nib = (w >> (4 * e)) & 0xFu;
+        const uint32_t tab = nib < 4 ? kI4E4m3Lo0 : nib < 8 ? kI4E4m3Lo1 : nib < 12 ? kI4E4m3Hi0 : kI4E4m3Hi1;
+        b[e] = (tab >> (8 * (nib & 3))) & 0xFFu;
+      }
+      out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+      out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
     }
     *reinterpret_cast<uint2*>(qw8 + static_cast<size_t>(n) * K + 8 * j) = out;
   }
-  const size_t pairs = static_cast<size_t>(K / 64) * n_pad;
-  if (i < pairs) {
-    const float s = __half2float(sw[i]);
-    float* f = reinterpret_cast<float*>(swp);  // i = g * n_pad + n, n_pad even
-    const size_t b = 2 * (i & ~static_cast<size_t>(1)) + (i & 1);
-    f[b] = s;
-    f[b + 2] = -kI2FMagic * s;  // exact: an fp16 significand times 3 * 2^22
-  }
+  const size_t scales = static_cast<size_t>(K / 64) * n_pad;
+  if (i < scales) sw32[i] = __half2float(sw[i]);
 }
 
 __global__ void l1s_kernel(const uint16_t* __restrict__ L1, const float* __restrict__ inv, int K, int r, int r_pad,
@@ -229,8 +227,8 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
     quantize_weights_kernel<true><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
         W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw), 0);
     const size_t work = std::max(static_cast<size_t>(w->n_pad) * (K / 8), static_cast<size_t>(K / 64) * w->n_pad);
-    int4_unpack_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(
-        w->qw, static_cast<const __half*>(w->sw), N, K, w->n_pad, w->qw8, w->swp);
+    int4_e4m3_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(
+        w->qw, static_cast<const __half*>(w->sw), N, K, w->n_pad, w->qw8, w->sw32);
   }
   if (rp > 0) {
     const size_t n1 = static_cast<size_t>(rp) * K;
