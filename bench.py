@@ -224,7 +224,7 @@ def _gpu_layer(svdq, li, dev, seed):
         svdq.svdq_act_global_scale(w, X, g)
         gx = float(g.item())
     ws = svdq.alloc_workspace(w, M, dev)
-    sx_off = (M * K // 2 + 1023) // 1024 * 1024
+    sx_off = (svdq.svdq_act_codes_bytes(w, M) + 1023) // 1024 * 1024
     la_off = sx_off + (svdq.svdq_act_scale_bytes(w, M) + 1023) // 1024 * 1024
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     act_scale_bytes = M * K // 16 if prec == svdq.SVDQ_NVFP4 else M * (K // 64) * 2

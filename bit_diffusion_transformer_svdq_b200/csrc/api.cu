@@ -442,9 +442,16 @@ svdq_status svdq_w4a4_gemm_lora_up_dyn(const svdq_weights* w, const uint8_t* qx,
   return gemm_entry(w, qx, sx, 1.0f, x_amax, lora_act, M, pro, epi, Y, out_dtype, stream);
 }
 
+size_t svdq_act_codes_bytes(const svdq_weights* w, int32_t M) {
+  if (!w || M < 0 || w->desc.precision == SVDQ_AWQ_W4A16) return 0;
+  const size_t packed = static_cast<size_t>(M) * (w->desc.K / 2);
+  if (w->desc.precision != SVDQ_INT4) return packed;
+  return int4_q8_offset(M, w->desc.K) + static_cast<size_t>(M) * w->desc.K;
+}
+
 size_t svdq_workspace_bytes(const svdq_weights* w, int32_t M) {
   if (!w || M < 0) return 0;
-  const size_t qx = static_cast<size_t>(round_up(static_cast<int64_t>(M) * (w->desc.K / 2), 1024));
+  const size_t qx = static_cast<size_t>(round_up(static_cast<int64_t>(svdq_act_codes_bytes(w, M)), 1024));
   const size_t sx = static_cast<size_t>(round_up(static_cast<int64_t>(svdq_act_scale_bytes(w, M)), 1024));
   const size_t la = static_cast<size_t>(round_up(static_cast<int64_t>(M) * w->rank_pad * 4, 1024));
   return qx + sx + la + 1024;  // + the dynamic tensor scale's amax word
@@ -468,7 +475,7 @@ svdq_status forward_entry(const svdq_weights* w, const uint16_t* X, int32_t M, f
   if (reinterpret_cast<uintptr_t>(workspace) & 1023u) return SVDQ_ERR_ALIGNMENT;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint8_t* qx = ws;
-  uint8_t* sx = qx + round_up(static_cast<int64_t>(M) * (w->desc.K / 2), 1024);
+  uint8_t* sx = qx + round_up(static_cast<int64_t>(svdq_act_codes_bytes(w, M)), 1024);
   float* la = reinterpret_cast<float*>(sx + round_up(static_cast<int64_t>(svdq_act_scale_bytes(w, M)), 1024));
   float* amax_slot = reinterpret_cast<float*>(ws + need - 1024);
   const bool nvfp4 = w->desc.precision == SVDQ_NVFP4;

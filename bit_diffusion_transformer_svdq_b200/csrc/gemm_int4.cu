@@ -11,23 +11,20 @@
 //
 // sm_100a design, one CTA per 128 x 128 output tile (persistent over the
 // tile list):
-//   warp 0      TMA producer: per ring stage (128 K = two groups) the packed
-//               activation codes (128 rows x 64 B, 64-byte swizzled) and the
-//               prepared E4M3 weight codes (128 rows x 128 B, 128-byte
-//               swizzled); per tile one stage of lora_act / L2 (fp32); per
-//               group the tile's 128 fp32 s_w and 128 fp16 s_x into a ring
-//               of eight shared-memory entries (released with one arrival per
-//               epilogue warp).
-//   warps 2-3   converters: two rows per lane, turn the packed codes into
-//               E4M3 bytes in the 128-byte-swizzled layout of the MMA operand
-//               (a byte permute through a 16-entry table, natural K order).
+//   warp 0      TMA producer: per ring stage (128 K = two groups) the
+//               activation codes as E4M3 bytes (the copy the quantiser writes
+//               beside the packed codes) and the prepared E4M3 weight codes,
+//               128 rows x 128 B each, 128-byte swizzled; per tile one stage
+//               of lora_act / L2 (fp32); per group the tile's 128 fp32 s_w
+//               and 128 fp16 s_x into a ring of eight shared-memory entries
+//               (released with one arrival per epilogue warp).
 //   warp 1      TMEM owner and MMA issuer: per group two kind::f8f6f4 MMAs
 //               (K = 32) into one of four fp32 accumulators (128 columns
 //               each), so the MMAs run up to three groups ahead of the
 //               scaling; per tile four kind::tf32 MMAs of the lora-up into
 //               the next accumulator, as one more "group" of scale 1.
-//   warps 4-19  epilogue: warp e = w - 4 owns rows 32 (e % 4) .. + 31 (its
-//               TMEM lane quarter) and columns 32 (e / 4) .. + 31; per group
+//   warps 2-17  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM
+//               lane quarter) and columns 32 ((w - 2) / 4) .. + 31; per group
 //               it reads its products, frees the accumulator and adds
 //               RN(P s_w) s_x to its fp32 accumulator with packed two-wide
 //               multiplies and FMAs, the 32 column scales read as eight
@@ -51,14 +48,12 @@ namespace svdq {
 namespace {
 
 constexpr int kTileM = 128, kTileN = 128;
-constexpr int kI4Stages = 5;
-constexpr int kApBytes = kTileM * 64;    // packed activation codes of a stage: 128 K per row
-constexpr int kA8Bytes = kTileM * 128;   // the same codes as E4M3 bytes
+constexpr int kI4Stages = 6;
+constexpr int kA8Bytes = kTileM * 128;   // activation codes of a stage (E4M3): 128 K per row
 constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes (E4M3)
-constexpr int kI4StageBytes = kApBytes + kA8Bytes + kB8Bytes;  // 40 KB
-constexpr int kConvWarps = 2;  // each lane converts two rows (r, r + 64)
+constexpr int kI4StageBytes = kA8Bytes + kB8Bytes;  // 32 KB
 constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
-constexpr int kI4Threads = 32 * (2 + kConvWarps + kI4EpiWarps);
+constexpr int kI4Threads = 32 * (2 + kI4EpiWarps);
 constexpr int kAccBufs = 4;  // fp32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
 constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
 // Group scales reach the epilogue through a ring of kScaleSlots entries in
@@ -77,27 +72,6 @@ static_assert(kI4Smem <= 232448, "shared memory budget");
 constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 // kind::tf32: fp32 D, tf32 A and B, K-major, N = 128, M = 128.
 constexpr uint32_t kIdescTf32x = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
-// Eight packed two's-complement codes (element e in bits 4e .. 4e+3) to
-// eight E4M3 bytes in the same order.  A byte permute looks each nibble's
-// low three bits up in the tables of n = 0..7 and n = 8..15; a second
-// permute spreads each nibble's bit 3 to a byte mask (the top bit of byte j
-// of w is bit 3 of nibble 2j + 1, that of byte j of w << 4 bit 3 of nibble
-// 2j) that picks between the two.
-__device__ __forceinline__ uint2 e4m3x8(uint32_t w) {
-  const uint32_t w4 = w << 4;
-  const uint32_t s0 = w & 0x7777u, s1 = (w >> 16) & 0x7777u;
-  const uint32_t m0 = prmt(w4, w, 0xD9C8u), m1 = prmt(w4, w, 0xFBEAu);
-  const uint32_t lo0 = prmt(kI4E4m3Lo0, kI4E4m3Lo1, s0), hi0 = prmt(kI4E4m3Hi0, kI4E4m3Hi1, s0);
-  const uint32_t lo1 = prmt(kI4E4m3Lo0, kI4E4m3Lo1, s1), hi1 = prmt(kI4E4m3Hi0, kI4E4m3Hi1, s1);
-  return make_uint2((hi0 & m0) | (lo0 & ~m0), (hi1 & m1) | (lo1 & ~m1));
-}
 
 struct I4Params {
   const __half* sx;   // [K/64][m_pad]
@@ -122,15 +96,14 @@ struct I4Params {
 
 template <bool kF32Out, bool kQkv>
 __global__ void __launch_bounds__(kI4Threads, 1)
-    gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_ap, const __grid_constant__ CUtensorMap tm_b8,
+    gemm_int4_kernel(const __grid_constant__ CUtensorMap tm_a8, const __grid_constant__ CUtensorMap tm_b8,
                      const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_lb,
                      const I4Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_s = reinterpret_cast<float*>(smem + kI4RedOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
-  uint64_t* conv = full + kI4Stages;      // activation codes unpacked (one arrival per converter warp)
-  uint64_t* empty = conv + kI4Stages;     // MMAs done with the stage
+  uint64_t* empty = full + kI4Stages;     // MMAs done with the stage
   uint64_t* acc_full = empty + kI4Stages;      // [kAccBufs]
   uint64_t* acc_empty = acc_full + kAccBufs;   // [kAccBufs], one arrival per epilogue warp
   uint64_t* sc_full = acc_empty + kAccBufs;    // [kScaleSlots], bulk copies of a group's scales
@@ -150,7 +123,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kI4Stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&conv[s], kConvWarps);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < kAccBufs; ++b) {
@@ -176,7 +148,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   // kernel; every global-memory access comes after this wait (the
   // descriptors are kernel parameters: their fetch may start before it)
   if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_ap);
+    prefetch_tmap(&tm_a8);
     prefetch_tmap(&tm_b8);
   }
   grid_dep_wait();
@@ -196,15 +168,14 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) goto teardown;
         if (elect_one()) {
           uint8_t* st = smem + stage * kI4StageBytes;
-          if (kb < num_kb) {  // packed activation codes, prepared weight codes
-            mbar_arrive_expect_tx(&full[stage], kApBytes + kB8Bytes);
-            tma_load_2d(st, &tm_ap, kb * 64, m0, &full[stage]);
-            tma_load_2d(st + kApBytes + kA8Bytes, &tm_b8, kb * 128, n0, &full[stage]);
+          mbar_arrive_expect_tx(&full[stage], kA8Bytes + kB8Bytes);
+          if (kb < num_kb) {  // activation and weight codes (E4M3)
+            tma_load_2d(st, &tm_a8, kb * 128, m0, &full[stage]);
+            tma_load_2d(st + kA8Bytes, &tm_b8, kb * 128, n0, &full[stage]);
           } else {  // lora_act and L2 columns 32 j .. 32 j + 31 (fp32)
             const int j = kb - num_kb;
-            mbar_arrive_expect_tx(&full[stage], kA8Bytes + kB8Bytes);
-            tma_load_2d(st + kApBytes, &tm_la, 32 * j, m0, &full[stage]);
-            tma_load_2d(st + kApBytes + kA8Bytes, &tm_lb, 32 * j, n0, &full[stage]);
+            tma_load_2d(st, &tm_la, 32 * j, m0, &full[stage]);
+            tma_load_2d(st + kA8Bytes, &tm_lb, 32 * j, n0, &full[stage]);
           }
         }
         __syncwarp();
@@ -233,52 +204,16 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         }
       }
     }
-  } else if (warp >= 2 && warp < 2 + kConvWarps) {
-    // ------------------------------------------------------- converters
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
-        if (kb < num_kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) goto teardown;
-#pragma unroll 1
-          for (int rr = 0; rr < kTileM / (32 * kConvWarps); ++rr) {
-            const int r = (rr * kConvWarps + warp - 2) * 32 + lane;  // row of the tile
-            // packed codes, 64-byte swizzled: row r's 16-byte unit j at r * 64 + ((j ^ ((r >> 1) & 3)) << 4)
-            const uint8_t* ap = smem + stage * kI4StageBytes + r * 64;
-            uint8_t* a8 = smem + stage * kI4StageBytes + kApBytes + r * 128;
-            uint4 in[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) in[j] = *reinterpret_cast<const uint4*>(ap + ((j ^ ((r >> 1) & 3)) << 4));
-            const uint32_t w[16] = {in[0].x, in[0].y, in[0].z, in[0].w, in[1].x, in[1].y, in[1].z, in[1].w,
-                                    in[2].x, in[2].y, in[2].z, in[2].w, in[3].x, in[3].y, in[3].z, in[3].w};
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {  // 16 codes: k = 16 u .. 16 u + 15
-              const uint2 b0 = e4m3x8(w[2 * u]), b1 = e4m3x8(w[2 * u + 1]);
-              *reinterpret_cast<uint4*>(a8 + ((u ^ (r & 7)) << 4)) = make_uint4(b0.x, b0.y, b1.x, b1.y);
-            }
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&conv[stage]);
-        }
-        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
-      }
-    }
   } else if (warp == 1) {
     // --------------------------------------------- MMA issuer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
-    // conv[s] completes once per K stage of slot s only (lora stages skip the
-    // converters), so its parity is tracked per slot, not with the ring phase
-    uint32_t conv_par = 0;
     uint32_t gcount = 0;  // accumulator uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb) {
-        if (!mbar_wait_warp(&conv[stage], (conv_par >> stage) & 1u, abort_flag)) goto teardown;
-        conv_par ^= 1u << stage;
+        if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + stage * kI4StageBytes + kApBytes);
+        const uint32_t sa = smem_u32(smem + stage * kI4StageBytes);
         const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
         const int ng = min(2, groups - 2 * kb);
         for (int gi = 0; gi < ng; ++gi, ++gcount) {
@@ -304,7 +239,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t sa = smem_u32(smem + stage * kI4StageBytes + kApBytes);
+            const uint32_t sa = smem_u32(smem + stage * kI4StageBytes);
             const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
@@ -321,16 +256,17 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
   } else {
     // ---------------------------------------------------------- epilogue
-    // warp e = 0..15 owns rows 32 (e % 4) .. + 31 (its TMEM lane quarter)
-    // and columns 32 (e / 4) .. + 31.  Per group it reads its 32 products
+    // warp w = 2..17 owns rows 32 (w % 4) .. + 31 (its TMEM lane quarter)
+    // and columns 32 ((w - 2) / 4) .. + 31.  Per group it reads its 32 products
     // (fp32: exact integers), frees the accumulator (one arrival per warp)
     // and adds RN(P s_w) s_x to its fp32 accumulator in registers.  The
     // group's scales come from the producer's ring (waited for per warp,
     // released with one arrival per warp): the warps never wait for one
     // another.
-    const int e = warp - 2 - kConvWarps;
-    const int q4 = e & 3;
-    const int cs = e >> 2;                  // column slice
+    // a warp reaches only the TMEM lanes of its rank in its warpgroup
+    // (warp % 4); the four warps 2 + 4c .. 5 + 4c cover the four quarters
+    const int q4 = warp & 3;
+    const int cs = (warp - 2) >> 2;         // column slice
     const int r = 32 * q4 + lane;           // row within the tile
     uint32_t gcount = 0;
     uint32_t sc_use = 0;  // scale-ring entries consumed
@@ -509,17 +445,18 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
                              void* Y, int out_dtype, const svdq_qkv_prologue* pro, cudaStream_t s) {
   const int K = w->desc.K, N = w->desc.N;
   const int m_pad = static_cast<int>(m_pad_of(M));
-  CUtensorMap tm_ap, tm_la;
-  // packed codes: M rows of K/2 bytes, 64-byte swizzled boxes of 128 rows x 64 bytes (128 K)
-  if (!encode_tmap_2d_swizzle(&tm_ap, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx, K / 2, M, K / 2, 64, kTileM,
-                              CU_TENSOR_MAP_SWIZZLE_64B))
+  CUtensorMap tm_a8, tm_la;
+  // the codes' E4M3 copy after the packed codes: M rows of K bytes, 128-byte
+  // swizzled boxes of 128 rows x 128 bytes (128 K)
+  if (!encode_tmap_2d_swizzle(&tm_a8, CU_TENSOR_MAP_DATA_TYPE_UINT8, qx + int4_q8_offset(M, K), K, M, K, 128, kTileM,
+                              CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (w->rank_pad > 0) {
     if (!encode_tmap_2d(&tm_la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, lora_act, w->rank_pad, M,
                         static_cast<uint64_t>(w->rank_pad) * 4, 32, kTileM))
       return cudaErrorInvalidValue;
   } else {
-    tm_la = tm_ap;  // unused without a low-rank branch
+    tm_la = tm_a8;  // unused without a low-rank branch
   }
   I4Params p;
   p.sx = static_cast<const __half*>(sx);
@@ -558,7 +495,7 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_ap, w->tm_qw8, tm_la, w->tm_l2, p);
+  return cudaLaunchKernelEx(&cfg, kern, tm_a8, w->tm_qw8, tm_la, w->tm_l2, p);
 }
 
 }  // namespace svdq

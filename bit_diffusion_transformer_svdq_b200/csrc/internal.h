@@ -23,6 +23,11 @@ inline int64_t m_pad_of(int64_t m) { return round_up(m, 128); }
 inline size_t nvfp4_scale_bytes(int64_t rows_padded, int K) { return static_cast<size_t>(rows_padded) * (K / 16); }
 inline size_t int4_scale_bytes(int64_t rows_padded, int K) { return static_cast<size_t>(rows_padded) * (K / 64) * 2; }
 
+// INT4 activation codes: the packed codes (M x K/2 bytes) are followed, at
+// this 1024-aligned offset of the same buffer, by the codes as E4M3 bytes
+// (M x K), the A operand of the INT4 GEMM.
+inline size_t int4_q8_offset(int64_t M, int K) { return static_cast<size_t>(round_up(M * (K / 2), 1024)); }
+
 // Offsets (bytes) of the sub-buffers inside the caller's weight storage.
 struct WeightLayout {
   size_t qw, sw, l1s, l2, inv_lambda, bias, status, amax, total;

@@ -103,6 +103,7 @@ _SIGS = {
     "svdq_act_global_scale": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_amax": (_I, [_P, _P, _I, _P, _P]),
     "svdq_act_scale_bytes": (_Z, [_P, _I]),
+    "svdq_act_codes_bytes": (_Z, [_P, _I]),
     "svdq_quantize_act_lora_down": (_I, [_P, _P, _I, _F, _P, _P, _P, _P]),
     "svdq_quantize_act_lora_down_dyn": (_I, [_P, _P, _I, _P, _P, _P, _P, _P]),
     "svdq_w4a4_gemm_lora_up": (_I, [_P, _P, _P, _F, _P, _I, _P, _I, _P]),
@@ -259,6 +260,10 @@ def svdq_act_amax(w: Weights, X: torch.Tensor, amax: torch.Tensor, stream=None) 
 
 def svdq_act_scale_bytes(w: Weights, M: int) -> int:
     return load_library().svdq_act_scale_bytes(w.handle, M)
+
+
+def svdq_act_codes_bytes(w: Weights, M: int) -> int:
+    return load_library().svdq_act_codes_bytes(w.handle, M)
 
 
 def svdq_workspace_bytes(w: Weights, M: int) -> int:

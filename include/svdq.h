@@ -247,6 +247,18 @@ SVDQ_API svdq_status svdq_act_global_scale(const svdq_weights* w, const uint16_t
  * value svdq_act_global_scale writes.  X [device] M x K bf16, M >= 1. */
 SVDQ_API svdq_status svdq_act_amax(const svdq_weights* w, const uint16_t* X, int32_t M, float* amax, void* stream);
 
+/* Bytes of the activation code buffer qx for M rows (0 for awq_w4a16
+ * weights, which quantise no activations):
+ *   NVFP4: M * K/2, the packed codes;
+ *   INT4:  the packed codes (M * K/2 bytes), then, from byte offset
+ *          round_up(M * K/2, 1024), the same codes as E4M3 bytes (M x K,
+ *          row-major, code k of row m at m * K + k): every integer in
+ *          [-8, 7] is exact in E4M3, and this copy is the INT4 GEMM's
+ *          tensor-core operand.
+ * svdq_quantize_act_lora_down writes the whole buffer and
+ * svdq_w4a4_gemm_lora_up reads it: allocate this many bytes. */
+SVDQ_API size_t svdq_act_codes_bytes(const svdq_weights* w, int32_t M);
+
 /* Bytes of the activation scale buffer sx for M rows:
  * NVFP4: ceil(M/128)*128 * K/16 (tiled layout); INT4: 2 * K/64 * ceil(M/128)*128. */
 SVDQ_API size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M);
@@ -263,7 +275,8 @@ SVDQ_API size_t svdq_act_scale_bytes(const svdq_weights* w, int32_t M);
  *   lora_act[m,t] = sum_k X[m,k] * L1s[t,k] (fp32 accumulation), then
  *     multiplied by RN32(1 / RN32(g_x * g_w)) (NVFP4; 1 for INT4) and
  *     rounded to tf32 (10-bit mantissa): the unit of the GEMM accumulator.
- * X [device] M x K bf16.  Outputs [device]: qx M x K/2 bytes; sx
+ * X [device] M x K bf16.  Outputs [device]: qx svdq_act_codes_bytes(w, M)
+ * bytes (the packed codes; for INT4 also their E4M3 copy); sx
  * svdq_act_scale_bytes(w, M) bytes (padding rows are written with zeros);
  * lora_act M x rank_pad fp32 (may be NULL when rank == 0). */
 SVDQ_API svdq_status svdq_quantize_act_lora_down(const svdq_weights* w, const uint16_t* X, int32_t M, float g_x,
@@ -287,7 +300,8 @@ SVDQ_API svdq_status svdq_quantize_act_lora_down_dyn(const svdq_weights* w, cons
  *                                 + lora_act L2^T) + b
  *   INT4:  Y = sum_g s_x s_w sum_{k in g} qx qw + lora_act L2^T + b
  * stored as bf16 (RNE) or fp32 (out_dtype).  Inputs as written by
- * svdq_quantize_act_lora_down.  Y [device] M x N. */
+ * svdq_quantize_act_lora_down: qx is the whole svdq_act_codes_bytes(w, M)
+ * buffer (INT4 reads only its E4M3 copy).  Y [device] M x N. */
 SVDQ_API svdq_status svdq_w4a4_gemm_lora_up(const svdq_weights* w, const uint8_t* qx, const void* sx, float g_x,
                                    const float* lora_act, int32_t M, void* Y, int32_t out_dtype, void* stream);
 

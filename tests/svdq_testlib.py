@@ -99,7 +99,7 @@ def gpu_prepare(svdq, li: synth.LayerInputs, ol: OracleLayer, precision: str | N
 def gpu_quantize(svdq, w, x_bits: np.ndarray, gx: float):
     M, K = x_bits.shape
     X = dev_u16(x_bits)
-    qx = aligned_empty(M * K // 2)
+    qx = aligned_empty(max(svdq.svdq_act_codes_bytes(w, M), 16))
     sx = aligned_empty(max(svdq.svdq_act_scale_bytes(w, M), 16))
     rp = w.view().rank_pad
     la = torch.empty((M, rp), dtype=torch.float32, device="cuda") if rp else None
@@ -175,6 +175,13 @@ def expected_act(x: np.ndarray, prep: V.Prepared, gx) -> dict:
     return dict(precision=prep.precision, qx=F.pack_nibbles(qx), sx=sx, lora_act=act.lora_act, act=act)
 
 
+def e4m3_bytes(codes: np.ndarray) -> np.ndarray:
+    """The E4M3 (fn) bytes of integer codes in [-8, 7], each exactly
+    representable, through torch's own float8 conversion."""
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
 def check_act_exact(svdq, w, x: np.ndarray, ol: OracleLayer, qx, sx, la, exp: dict | None = None) -> dict:
     """Activation codes and scales of every row bit-exact against the
     oracle's quantiser (scales exported in canonical layout through the C
@@ -185,6 +192,11 @@ def check_act_exact(svdq, w, x: np.ndarray, ol: OracleLayer, qx, sx, la, exp: di
         exp = expected_act(x, ol.prep, ol.gx)
     precision = exp["precision"]
     assert np.array_equal(qx[:M * K // 2].cpu().numpy().reshape(M, K // 2), exp["qx"])
+    if precision == "int4":
+        # the same codes as E4M3 bytes, M rows of K, at the end of the codes buffer
+        nb = svdq.svdq_act_codes_bytes(w, M)
+        q8 = qx[nb - M * K:nb].cpu().numpy().reshape(M, K)
+        assert np.array_equal(q8, e4m3_bytes(exp["act"].qx))
     sc = svdq.svdq_export_act_scales(w, sx, M)
     assert np.array_equal(sc if precision == "nvfp4" else sc.view(np.uint16), exp["sx"])
     mp = (M + 127) // 128 * 128

@@ -88,14 +88,14 @@ def test_dyn_quantize_bit_exact(svdq, name, a_over, b_over):
     X = T.dev_u16(li.x_bits)
     a = torch.empty(1, dtype=torch.float32, device="cuda")
     svdq.svdq_act_amax(w, X, a)
-    qx = T.aligned_empty(M * K // 2)
+    qx = T.aligned_empty(svdq.svdq_act_codes_bytes(w, M))
     sx = T.aligned_empty(svdq.svdq_act_scale_bytes(w, M))
     rp = w.view().rank_pad
     la = torch.empty((M, rp), dtype=torch.float32, device="cuda")
     svdq.svdq_quantize_act_lora_down_dyn(w, X, M, a, qx, sx, la)
     torch.cuda.synchronize()
     act = V.quantize_activations(li.x, ol.prep, ol.gx)
-    assert np.array_equal(T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2)), act.qx)
+    assert np.array_equal(T.unpack_codes(qx[:M * K // 2].cpu().numpy().reshape(M, K // 2)), act.qx)
     assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K), act.sx)
     # lora_act: the same buffer as the static call with the same g_x (bit for bit)
     X2, qx2, sx2, la2 = T.gpu_quantize(svdq, w, li.x_bits, float(ol.gx))
@@ -205,7 +205,7 @@ def test_nonfinite_dynamic_scale_sets_status(svdq):
     w = T.gpu_prepare(svdq, li, ol)
     M, K = 64, 256
     a = torch.full((1,), float("inf"), dtype=torch.float32, device="cuda")
-    qx = T.aligned_empty(M * K // 2)
+    qx = T.aligned_empty(svdq.svdq_act_codes_bytes(w, M))
     sx = T.aligned_empty(svdq.svdq_act_scale_bytes(w, M))
     la = torch.empty((M, w.view().rank_pad), dtype=torch.float32, device="cuda")
     svdq.svdq_quantize_act_lora_down_dyn(w, T.dev_u16(li.x_bits), M, a, qx, sx, la)

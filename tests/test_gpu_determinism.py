@@ -54,7 +54,7 @@ def test_repeated_calls_are_bit_identical(svdq, workload, seed, precision):
     rp = w.view().rank_pad
     first = None
     for _ in range(REPEATS):
-        qx = torch.empty(M * K // 2, dtype=torch.uint8, device="cuda")
+        qx = torch.empty(svdq.svdq_act_codes_bytes(w, M), dtype=torch.uint8, device="cuda")
         sx = T.aligned_empty(svdq.svdq_act_scale_bytes(w, M))
         la = torch.empty((M, rp), dtype=torch.float32, device="cuda")
         # poison the outputs: nothing may be left over from a previous call

@@ -104,7 +104,7 @@ def test_act_global_scale_bit_exact(svdq):
 def _check_act_codes(svdq, w, li, ol, qx, sx, la, precision):
     M, K = li.shape.M, li.shape.K
     act = V.quantize_activations(li.x, ol.prep, ol.gx)
-    got_codes = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
+    got_codes = T.unpack_codes(qx[:M * K // 2].cpu().numpy().reshape(M, K // 2))
     if precision == "nvfp4":
         assert np.array_equal(got_codes, act.qx)
         sxh = sx.cpu().numpy()
@@ -114,6 +114,9 @@ def _check_act_codes(svdq, w, li, ol, qx, sx, la, precision):
         assert np.all(sxh[pad] == 0)
     else:
         assert np.array_equal(T.nibbles_to_int(got_codes), act.qx)
+        # the E4M3 copy of the codes the GEMM reads, after the packed codes
+        nb = svdq.svdq_act_codes_bytes(w, M)
+        assert np.array_equal(qx[nb - M * K:nb].cpu().numpy().reshape(M, K), T.e4m3_bytes(act.qx))
         mp = (M + 127) // 128 * 128
         sxh = sx.cpu().numpy().view(np.float16).reshape(K // 64, mp)
         assert np.array_equal(sxh[:, :M].T.view(np.uint16), act.sx.view(np.uint16))
@@ -173,7 +176,7 @@ def test_quantize_rounding_ties_and_signed_zero(svdq):
     X, qx, sx, la = T.gpu_quantize(svdq, w_gpu, x_bits, 1.0)
     act = V.quantize_activations(x, ol.prep, gx)
     assert np.any(act.qx == 8)  # -0 codes are present
-    got = T.unpack_codes(qx.cpu().numpy().reshape(M, K // 2))
+    got = T.unpack_codes(qx[:M * K // 2].cpu().numpy().reshape(M, K // 2))
     assert np.array_equal(got, act.qx)
     assert np.array_equal(T.untile_nvfp4_scales(sx.cpu().numpy(), M, K), act.sx)
 
@@ -259,9 +262,10 @@ def test_forward_parity_int4(svdq, name, wl, over, out_dtype):
 def test_int4_gemm_exact_on_integer_grid(svdq):
     """INT4 counterpart of the exactness pin: lambda = 1, rank 0, integer
     codes and power-of-two fp16 scales make every partial sum an fp32-exact
-    value, so the kind::i8 product with its per-group scaling must equal the
-    oracle bit for bit.  This pins the nibble unpacking, the K permutation
-    inside 8-value blocks (the same on both operands) and both scale layouts.
+    value, so the kind::f8f6f4 product of the E4M3 codes with its per-group
+    scaling must equal the oracle bit for bit.  This pins the E4M3 copies of
+    both operands (the activations' written here from the definition, after
+    the packed codes in the same buffer) and both scale layouts.
     K = 576 is an odd number of 64-groups (a half-filled last ring stage)."""
     rng = np.random.default_rng(9)
     M, K, N = 200, 576, 320
@@ -281,7 +285,11 @@ def test_int4_gemm_exact_on_integer_grid(svdq):
     mp = (M + 127) // 128 * 128
     sx_dev = np.zeros((K // 64, mp), np.float16)
     sx_dev[:, :M] = sx.T
-    qx = torch.from_numpy(F.pack_nibbles((codes.astype(np.int16) & 0xF).astype(np.uint8))).cuda()
+    nb = svdq.svdq_act_codes_bytes(w, M)
+    buf = np.zeros(nb, np.uint8)
+    buf[:M * K // 2] = F.pack_nibbles((codes.astype(np.int16) & 0xF).astype(np.uint8)).ravel()
+    buf[nb - M * K:] = T.e4m3_bytes(codes).ravel()
+    qx = torch.from_numpy(buf).cuda()
     sxt = torch.from_numpy(sx_dev.view(np.uint16).astype(np.int16)).cuda()
     Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
     svdq.svdq_w4a4_gemm_lora_up(w, qx, sxt, 1.0, None, M, Y, 1)
