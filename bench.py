@@ -64,7 +64,13 @@ def _peaks():
 
 
 def _src_hash(path):
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    """Hash of a kernel's source file together with the shared device
+    headers it includes (a change to either changes the kernel)."""
+    h = hashlib.sha256()
+    d = os.path.dirname(path)
+    for f in (path, os.path.join(d, "ptx.cuh"), os.path.join(d, "internal.h")):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
 
 
 def _traffic(key, src):
