@@ -3,11 +3,16 @@
 // tcgen05 has no 4-bit integer kind, so the codes go to the tensor core as
 // 8-bit operands: E4M3 bytes, which hold every integer in [-8, 7] exactly,
 // multiplied by kind::f8f6f4 MMAs into fp32 TMEM accumulators.  Every
-// product is an integer of magnitude at most 64 and a group's sum at most
-// 4096, so the accumulator holds each group's integer dot product exactly,
-// as a float; the scales change with every 64-group, so each group's
-// product leaves TMEM and is scaled into an fp32 accumulator held in
-// registers: acc += RN(P s_w) s_x.
+// product is an integer of magnitude at most 64 and a group's sum P at most
+// 4096, so the accumulator holds each group's integer dot product exactly.
+// The scales change with every 64-group, so each group's product leaves TMEM
+// and is added into an fp32 accumulator held in registers.  The tensor core
+// also forms the group's scale products C[m,n] = s_x[m,g] s_w[n,g]: one
+// kind::f16 MMA whose operands are zero but for their first K row (s_x and
+// s_w, both fp16), which gives the 22-bit products exactly.  The epilogue
+// then takes one FMA per element and group, acc = RN(P C + acc): the same
+// single rounding as acc = RN(RN(P s_w) s_x + acc), since P s_w (at most
+// 13 x 11 significant bits) is exact in fp32.
 //
 // sm_100a design, one CTA per 128 x 128 output tile (persistent over the
 // tile list):
@@ -15,27 +20,23 @@
 //               activation codes as E4M3 bytes (the copy the quantiser writes
 //               beside the packed codes) and the prepared E4M3 weight codes,
 //               128 rows x 128 B each, 128-byte swizzled; per tile one stage
-//               of lora_act / L2 (fp32); per group the tile's 128 fp32 s_w
-//               and 128 fp16 s_x into a ring of eight shared-memory entries
-//               (released with one arrival per epilogue warp).
+//               of lora_act / L2 (fp32); per group the tile's 128 fp16 s_x
+//               and 128 fp16 s_w into the first K row of a scale slot (four
+//               128-byte bulk copies).
 //   warp 1      TMEM owner and MMA issuer: per group two kind::f8f6f4 MMAs
-//               (K = 32) into one of four fp32 accumulators (128 columns
-//               each), so the MMAs run up to three groups ahead of the
-//               scaling; per tile four kind::tf32 MMAs of the lora-up into
-//               the next accumulator, as one more "group" of scale 1.
+//               (K = 32) into P and one kind::f16 MMA (K = 16, MN-major
+//               operands from the scale slot) into C, in one of two buffers
+//               of 256 columns (P, C); per tile four kind::tf32 MMAs of the
+//               lora-up into the next buffer's P, as one more "group".
 //   warps 2-17  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM
 //               lane quarter) and columns 32 ((w - 2) / 4) .. + 31; per group
-//               it reads its products, frees the accumulator and adds
-//               RN(P s_w) s_x to its fp32 accumulator with packed two-wide
-//               multiplies and FMAs, the 32 column scales read as eight
-//               broadcast 16-byte loads.  Finally y = acc + b is stored; the
-//               QKV variant first applies the attention prologue (per
-//               128-column head of Q and K: RMS normalisation, weight, rotary
-//               embedding), the four column slices of a row adding their sums
-//               of squares through shared memory.
-// The group rescale is CUDA-core work on every output element (one packed
-// multiply and one packed FMA per two elements per 64 K, against 64 MACs on
-// the tensor core), so this kernel is bound by it, not by the MMAs.
+//               it loads P and C in two halves of 16 columns, frees the
+//               buffer and adds P C into its fp32 accumulator with packed
+//               two-wide FMAs.  Finally y = acc + b is stored; the QKV variant
+//               first applies the attention prologue (per 128-column head of
+//               Q and K: RMS normalisation, weight, rotary embedding), the
+//               four column slices of a row adding their sums of squares
+//               through shared memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -54,28 +55,34 @@ constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes (E4M3)
 constexpr int kI4StageBytes = kA8Bytes + kB8Bytes;  // 32 KB
 constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
 constexpr int kI4Threads = 32 * (2 + kI4EpiWarps);
-constexpr int kAccBufs = 4;  // fp32 group accumulators of 128 columns: the MMAs run up to 3 groups ahead
-constexpr uint32_t kI4TmemCols = 128 * kAccBufs;
-// Group scales reach the epilogue through a ring of kScaleSlots entries in
-// shared memory, filled by the producer with bulk copies: per entry the
-// tile's 128 fp32 s_w and its 128 fp16 s_x.
-constexpr int kScaleSlots = 8;
-constexpr int kScaleSlotBytes = kTileN * 4 + kTileM * 2;  // 768
+constexpr int kAccBufs = 2;      // group buffers of 256 TMEM columns: P (128) then C (128)
+constexpr uint32_t kI4TmemCols = 256 * kAccBufs;
+// Scale slots: the two operands of a group's C MMA, each an MN-major
+// 128-byte-swizzled tile of two 1 KB atoms (64 fp16 along M or N x K rows
+// 0-7); only row 0 of each atom is ever written (the group's scales), rows
+// 1-7 stay zero, and K rows 8-15 of every operand are one shared 2 KB block
+// of zeros (reached through the descriptor's K-group stride).
+constexpr int kScaleSlots = 6;
+constexpr int kSlotBytes = 4096;  // s_x operand (2 KB), then s_w operand (2 KB)
 constexpr int kScaleOff = kI4Stages * kI4StageBytes;
-constexpr int kI4BarOff = kScaleOff + kScaleSlots * kScaleSlotBytes;
+constexpr int kZeroOff = kScaleOff + kScaleSlots * kSlotBytes;
+constexpr int kI4BarOff = kZeroOff + 2048;
 constexpr int kI4RedOff = kI4BarOff + 512;  // QKV: one float per row and column slice (16 x 32)
 constexpr size_t kI4Smem = kI4RedOff + kI4EpiWarps * 32 * 4 + 1024 /*align*/;
-static_assert(kI4StageBytes % 1024 == 0, "stages keep 1024-byte alignment");
+static_assert(kI4StageBytes % 1024 == 0 && kScaleOff % 1024 == 0 && kZeroOff % 1024 == 0, "1 KB atoms");
 static_assert(kI4Smem <= 232448, "shared memory budget");
 
 // kind::f8f6f4: fp32 D, E4M3 A and B, K-major, N = 128, M = 128.
 constexpr uint32_t kIdescF8 = (1u << 4) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
+// kind::f16: fp32 D, fp16 A and B, both MN-major, N = 128, M = 128.
+constexpr uint32_t kIdescScale =
+    (1u << 4) | (1u << 15) | (1u << 16) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 // kind::tf32: fp32 D, tf32 A and B, K-major, N = 128, M = 128.
 constexpr uint32_t kIdescTf32x = (1u << 4) | (2u << 7) | (2u << 10) | (uint32_t(kTileN >> 3) << 17) | (uint32_t(kTileM >> 4) << 24);
 
 struct I4Params {
   const __half* sx;   // [K/64][m_pad]
-  const float* sw32;  // [K/64][n_pad]
+  const __half* sw;   // [K/64][n_pad]
   const float* bias;
   void* Y;
   int* status;
@@ -89,9 +96,6 @@ struct I4Params {
   const float* rope_sin;
   float eps;
   int qk_cols;  // 2 * heads * 128; K starts at qk_cols / 2
-  // 0 at run time, unknown to the compiler: ANDing a loaded value with it
-  // gives a zero that still depends on the load (see the scale release)
-  uint32_t dep_mask;
 };
 
 template <bool kF32Out, bool kQkv>
@@ -103,11 +107,11 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* red_s = reinterpret_cast<float*>(smem + kI4RedOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kI4BarOff);
-  uint64_t* empty = full + kI4Stages;     // MMAs done with the stage
+  uint64_t* empty = full + kI4Stages;          // MMAs done with the stage
   uint64_t* acc_full = empty + kI4Stages;      // [kAccBufs]
   uint64_t* acc_empty = acc_full + kAccBufs;   // [kAccBufs], one arrival per epilogue warp
   uint64_t* sc_full = acc_empty + kAccBufs;    // [kScaleSlots], bulk copies of a group's scales
-  uint64_t* sc_empty = sc_full + kScaleSlots;  // [kScaleSlots], one arrival per epilogue warp
+  uint64_t* sc_empty = sc_full + kScaleSlots;  // [kScaleSlots], the C MMA that read the slot is done
   uint64_t* drain = sc_empty + kScaleSlots;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -120,6 +124,11 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   const int groups = p.K / 64;
   const int num_kb = (groups + 1) / 2;  // ring stages per tile (the last may hold one group)
 
+  // the scale slots and the shared K rows 8-15 start (and, but for the
+  // scale rows the copies write, stay) zero
+  for (int o = threadIdx.x * 16; o < kScaleSlots * kSlotBytes + 2048; o += kI4Threads * 16)
+    *reinterpret_cast<uint4*>(smem + kScaleOff + o) = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kI4Stages; ++s) {
       mbar_init(&full[s], 1);
@@ -131,7 +140,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     }
     for (int b = 0; b < kScaleSlots; ++b) {
       mbar_init(&sc_full[b], 1);
-      mbar_init(&sc_empty[b], kI4EpiWarps);
+      mbar_init(&sc_empty[b], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -155,13 +164,13 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   if (threadIdx.x == 0) grid_dep_launch();
   const uint32_t tmem = *tmem_slot;
   uint32_t issued_mask = 0, issued_par = 0;
-  uint32_t sc_mask = 0, sc_par = 0;  // scale-ring entries issued (teardown drain)
+  uint32_t sc_mask = 0, sc_par = 0;  // scale slots issued (teardown drain)
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t sc_count = 0;  // scale-ring entries issued so far
+    uint32_t sc_count = 0;  // scale slots filled so far
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
       for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
@@ -182,8 +191,8 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
-        // the scales of this stage's groups, one ring entry per group (after
-        // the operands, so that a slow epilogue never holds the MMAs back)
+        // the scales of this stage's groups, one slot per group: row 0 of the
+        // two atoms of each operand (64 fp16 = 128 bytes each)
         if (kb < num_kb) {
           const int ng = min(2, groups - 2 * kb);
           for (int gi = 0; gi < ng; ++gi, ++sc_count) {
@@ -192,10 +201,14 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             if (!mbar_wait_warp(&sc_empty[ss], sp ^ 1, abort_flag)) goto teardown;
             if (elect_one()) {
               const int g = 2 * kb + gi;
-              uint8_t* dst = smem + kScaleOff + ss * kScaleSlotBytes;
-              mbar_arrive_expect_tx(&sc_full[ss], kScaleSlotBytes);
-              bulk_load(dst, p.sw32 + static_cast<size_t>(g) * p.n_pad + n0, kTileN * 4, &sc_full[ss]);
-              bulk_load(dst + kTileN * 4, p.sx + static_cast<size_t>(g) * p.m_pad + m0, kTileM * 2, &sc_full[ss]);
+              uint8_t* dst = smem + kScaleOff + ss * kSlotBytes;
+              const __half* sxg = p.sx + static_cast<size_t>(g) * p.m_pad + m0;
+              const __half* swg = p.sw + static_cast<size_t>(g) * p.n_pad + n0;
+              mbar_arrive_expect_tx(&sc_full[ss], 512);
+              bulk_load(dst, sxg, 128, &sc_full[ss]);
+              bulk_load(dst + 1024, sxg + 64, 128, &sc_full[ss]);
+              bulk_load(dst + 2048, swg, 128, &sc_full[ss]);
+              bulk_load(dst + 3072, swg + 64, 128, &sc_full[ss]);
             }
             __syncwarp();
             sc_mask |= 1u << ss;
@@ -208,7 +221,9 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     // --------------------------------------------- MMA issuer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t gcount = 0;  // accumulator uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
+    uint32_t gcount = 0;  // buffer uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
+    uint32_t sc_use = 0;  // scale slots consumed
+    const uint32_t zero_blk = smem_u32(smem + kZeroOff);
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
@@ -216,15 +231,24 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         const uint32_t sa = smem_u32(smem + stage * kI4StageBytes);
         const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
         const int ng = min(2, groups - 2 * kb);
-        for (int gi = 0; gi < ng; ++gi, ++gcount) {
+        for (int gi = 0; gi < ng; ++gi, ++gcount, ++sc_use) {
+          const uint32_t ss = sc_use % kScaleSlots;
+          if (!mbar_wait_warp(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) goto teardown;
           const uint32_t buf = gcount % kAccBufs;
           if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
           tc_fence_after();
           if (elect_one()) {
+            const uint32_t d = tmem + buf * 256;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // K = 32 E4M3 (32 bytes) per MMA
-              mma_f8(tmem + buf * kTileN, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescF8, k ? 1u : 0u);
+              mma_f8(d, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescF8, k ? 1u : 0u);
+            // C = s_x s_w^T: MN-major operands, atoms 1 KB apart along M / N,
+            // K rows 8-15 in the shared zero block
+            const uint32_t sxa = smem_u32(smem + kScaleOff + ss * kSlotBytes), swa = sxa + 2048;
+            mma_bf16(d + 128, sdesc_sw128_mn(sxa, 1024, zero_blk - sxa), sdesc_sw128_mn(swa, 1024, zero_blk - swa),
+                     kIdescScale, 0u);
             tc_commit(&acc_full[buf]);
+            tc_commit(&sc_empty[ss]);
           }
           __syncwarp();
         }
@@ -232,7 +256,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         __syncwarp();
         if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
       }
-      if (p.n_lora > 0) {  // the lora-up as one more accumulator use, of scale 1
+      if (p.n_lora > 0) {  // the lora-up as one more buffer use (P only), of scale 1
         const uint32_t buf = gcount % kAccBufs;
         if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
         for (int j = 0; j < p.n_lora; ++j) {
@@ -243,7 +267,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
-              mma_tf32(tmem + buf * kTileN, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
+              mma_tf32(tmem + buf * 256, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
             tc_commit(&empty[stage]);
           }
           __syncwarp();
@@ -257,19 +281,18 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   } else {
     // ---------------------------------------------------------- epilogue
     // warp w = 2..17 owns rows 32 (w % 4) .. + 31 (its TMEM lane quarter)
-    // and columns 32 ((w - 2) / 4) .. + 31.  Per group it reads its 32 products
-    // (fp32: exact integers), frees the accumulator (one arrival per warp)
-    // and adds RN(P s_w) s_x to its fp32 accumulator in registers.  The
-    // group's scales come from the producer's ring (waited for per warp,
-    // released with one arrival per warp): the warps never wait for one
-    // another.
-    // a warp reaches only the TMEM lanes of its rank in its warpgroup
-    // (warp % 4); the four warps 2 + 4c .. 5 + 4c cover the four quarters
+    // and columns 32 ((w - 2) / 4) .. + 31.  Per group it reads its 32
+    // products P (fp32: exact integers) and scale products C in two halves,
+    // frees the buffer (one arrival per warp) and adds RN(P C + acc) into
+    // its fp32 accumulator in registers: the warps never wait for one
+    // another.  A warp reaches only the TMEM lanes of its rank in its
+    // warpgroup (warp % 4); the four warps 2 + 4c .. 5 + 4c cover the four
+    // quarters.
     const int q4 = warp & 3;
     const int cs = (warp - 2) >> 2;         // column slice
     const int r = 32 * q4 + lane;           // row within the tile
+    const uint32_t tq = tmem + (static_cast<uint32_t>(32 * q4) << 16) + 32 * cs;
     uint32_t gcount = 0;
-    uint32_t sc_use = 0;  // scale-ring entries consumed
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
@@ -280,55 +303,32 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       for (int c = 0; c < 32; ++c) acc[c] = 0.0f;
       const int uses = groups + (p.n_lora > 0 ? 1 : 0);
       for (int g = 0; g < uses; ++g, ++gcount) {
-        const uint32_t ss = sc_use % kScaleSlots;  // this group's ring entry
-        if (g < groups && !mbar_wait(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
         const uint32_t buf = gcount % kAccBufs;
         if (!mbar_wait(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        uint32_t P[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * q4) << 16) + buf * kTileN + 32 * cs, P);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acc_empty[buf]);  // the products are in registers: free the buffer
-        if (g < groups) {
-          // the warp's 32 column scales, eight broadcast 16-byte loads; two
-          // columns per packed multiply (RN(P s_w)) and packed FMA (+ s_x)
-          const uint8_t* sb = smem + kScaleOff + ss * kScaleSlotBytes;
-          const float sxr = __half2float(reinterpret_cast<const __half*>(sb + kTileN * 4)[r]);
-          const float4* sw4 = reinterpret_cast<const float4*>(sb) + 8 * cs;
-          const float2 sx2 = make_float2(sxr, sxr);
-          uint32_t dep = __float_as_uint(sxr);
+        const uint32_t tb = tq + buf * 256;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 t = ld_shared_f4_inorder(sw4 + q);
-            dep ^= __float_as_uint(t.x);
-            const float2 u0 = __fmul2_rn(make_float2(__uint_as_float(P[4 * q]), __uint_as_float(P[4 * q + 1])),
-                                         make_float2(t.x, t.y));
-            const float2 u1 = __fmul2_rn(make_float2(__uint_as_float(P[4 * q + 2]), __uint_as_float(P[4 * q + 3])),
-                                         make_float2(t.z, t.w));
-            const float2 a0 = __ffma2_rn(u0, sx2, make_float2(acc[4 * q], acc[4 * q + 1]));
-            const float2 a1 = __ffma2_rn(u1, sx2, make_float2(acc[4 * q + 2], acc[4 * q + 3]));
-            acc[4 * q] = a0.x;
-            acc[4 * q + 1] = a0.y;
-            acc[4 * q + 2] = a1.x;
-            acc[4 * q + 3] = a1.y;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t P[16], C[16];
+          tmem_ld16x2_wait(tb + 16 * h, tb + 128 + 16 * h, P, C);  // C is not read for the lora-up
+          if (h == 1) {  // both halves are in registers: free the buffer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[buf]);
           }
-          // Release the ring entry.  The producer's next bulk copy may then
-          // overwrite it, so the arrival must follow the completion of every
-          // load of the entry above: its address depends on one value of
-          // each load, through a zero the compiler cannot fold away (a
-          // run-time mask that is 0).
-          const uint32_t zero = dep & p.dep_mask;
-          __syncwarp();
-          if (lane == 0) mbar_arrive_at(smem_u32(&sc_empty[ss]) + zero);
-          ++sc_use;
-        } else {  // the lora-up, fp32
+          if (g < groups) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) acc[c] = __fadd_rn(acc[c], __uint_as_float(P[c]));
+            for (int c = 0; c < 16; c += 2) {
+              const float2 a = __ffma2_rn(make_float2(__uint_as_float(P[c]), __uint_as_float(P[c + 1])),
+                                          make_float2(__uint_as_float(C[c]), __uint_as_float(C[c + 1])),
+                                          make_float2(acc[16 * h + c], acc[16 * h + c + 1]));
+              acc[16 * h + c] = a.x;
+              acc[16 * h + c + 1] = a.y;
+            }
+          } else {  // the lora-up, fp32
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc[16 * h + c] = __fadd_rn(acc[16 * h + c], __uint_as_float(P[c]));
+          }
         }
       }
       if (!ok) break;
@@ -460,7 +460,7 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   }
   I4Params p;
   p.sx = static_cast<const __half*>(sx);
-  p.sw32 = w->sw32;
+  p.sw = static_cast<const __half*>(w->sw);
   p.bias = w->bias;
   p.Y = Y;
   p.status = w->status;
@@ -476,7 +476,6 @@ cudaError_t launch_gemm_int4(const svdq_weights* w, const uint8_t* qx, const voi
   p.rope_sin = pro ? pro->rope_sin : nullptr;
   p.eps = pro ? pro->eps : 0.0f;
   p.qk_cols = pro ? 2 * pro->heads * pro->head_dim : 0;
-  p.dep_mask = 0;
   const int tiles = ((M + kTileM - 1) / kTileM) * ((N + kTileN - 1) / kTileN);
   const int grid = std::min(tiles, num_sms(w->device));
   const bool f32 = out_dtype == SVDQ_OUT_F32;

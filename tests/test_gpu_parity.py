@@ -300,6 +300,71 @@ def test_int4_gemm_exact_on_integer_grid(svdq):
     assert np.array_equal(Y.cpu().numpy().astype(np.float64), ref)
 
 
+def _rn32(fr):
+    """fp32 round-to-nearest-even of an exact rational (normal range)."""
+    from fractions import Fraction
+    if fr == 0:
+        return np.float32(0.0)
+    a = abs(fr)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    scale = Fraction(2) ** (23 - e)  # a * scale in [2^23, 2^24)
+    x = a * scale
+    n = x.numerator // x.denominator
+    rem = x - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    v = np.float32(float(Fraction(n) / scale))
+    return -v if fr < 0 else v
+
+
+def test_int4_gemm_rounds_once_per_group(svdq):
+    """The INT4 GEMM's accumulation with arbitrary fp16 scales: for every
+    output, acc = RN32(P_g s_w s_x + acc) group after group (P_g the exact
+    integer group sum), one rounding per group, then + b (0 here).  The
+    expected values are exact rationals rounded to fp32 here, so fp32 Y
+    must match bit for bit.  Rank 0, lambda = 1, four groups."""
+    from fractions import Fraction
+    rng = np.random.default_rng(21)
+    M, K, N = 64, 256, 128
+    G = K // 64
+    s_w = (rng.uniform(0.5, 2.0, size=(N, G)) * 2.0 ** rng.integers(-6, 2, size=(N, G))).astype(np.float16)
+    q_w = rng.integers(-7, 8, size=(N, K))
+    q_w[:, ::64] = 7  # every group's amax is 7 s_w: the codes are W / s_w exactly
+    W = (q_w * np.repeat(s_w.astype(np.float32), 64, axis=1)).astype(np.float32)
+    li = synth.LayerInputs(synth.WORKLOADS["tiny"], 0, np.zeros((M, K), np.uint16), np.zeros((M, K), np.float32), W,
+                           T.bf16_bits(np.zeros(N)), np.zeros(N, np.float32))
+    ol = T.oracle_layer(li, precision="int4", rank=0, lam=np.ones(K, np.float32))
+    assert np.array_equal(ol.prep.qw.astype(np.int64), q_w)
+    assert np.array_equal(ol.prep.sw.view(np.uint16), s_w.view(np.uint16))
+    w = T.gpu_prepare(svdq, li, ol, "int4")
+    codes = rng.integers(-8, 8, size=(M, K)).astype(np.int8)
+    sx = (rng.uniform(0.5, 2.0, size=(M, G)) * 2.0 ** rng.integers(-6, 2, size=(M, G))).astype(np.float16)
+    mp = (M + 127) // 128 * 128
+    sx_dev = np.zeros((G, mp), np.float16)
+    sx_dev[:, :M] = sx.T
+    nb = svdq.svdq_act_codes_bytes(w, M)
+    buf = np.zeros(nb, np.uint8)
+    buf[:M * K // 2] = F.pack_nibbles((codes.astype(np.int16) & 0xF).astype(np.uint8)).ravel()
+    buf[nb - M * K:] = T.e4m3_bytes(codes).ravel()
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    svdq.svdq_w4a4_gemm_lora_up(w, torch.from_numpy(buf).cuda(),
+                                torch.from_numpy(sx_dev.view(np.uint16).astype(np.int16)).cuda(), 1.0, None, M, Y, 1)
+    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(w) == 0
+    y = Y.cpu().numpy()
+    P = np.einsum("mgk,ngk->mng", codes.astype(np.int64).reshape(M, G, 64), q_w.reshape(N, G, 64))
+    fw = [[Fraction(float(v)) for v in row] for row in s_w.astype(np.float64)]
+    fx = [[Fraction(float(v)) for v in row] for row in sx.astype(np.float64)]
+    for m in range(M):
+        for n in range(N):
+            acc = np.float32(0.0)
+            for g in range(G):
+                acc = _rn32(int(P[m, n, g]) * fw[n][g] * fx[m][g] + Fraction(float(acc)))
+            assert y[m, n].view(np.uint32) == acc.view(np.uint32), (m, n, y[m, n], acc)
+
+
 def test_argument_errors(svdq):
     li = _layer("tiny", {})
     ol = T.oracle_layer(li)
