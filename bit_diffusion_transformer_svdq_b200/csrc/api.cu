@@ -127,7 +127,6 @@ WeightLayout weight_layout(const svdq_layer_desc& d) {
   L.amax = take(16);
   if (d.precision == SVDQ_INT4) {
     L.qw8 = take(static_cast<size_t>(np) * d.K);
-    L.sw32 = take(static_cast<size_t>(d.K / 64) * np * 4);
   }
   L.total = off;
   return L;
@@ -243,7 +242,6 @@ svdq_status svdq_prepare_weights(const svdq_layer_desc* desc, const float* W, co
   w->status = reinterpret_cast<int*>(b + L.status);
   w->amax = reinterpret_cast<uint32_t*>(b + L.amax);
   w->qw8 = desc->precision == SVDQ_INT4 ? b + L.qw8 : nullptr;
-  w->sw32 = desc->precision == SVDQ_INT4 ? reinterpret_cast<float*>(b + L.sw32) : nullptr;
 
   bool ok = encode_tmap_2d(&w->tm_qw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->qw, desc->K / 2, desc->N, desc->K / 2, 128,
                            128);

@@ -20,9 +20,10 @@
 //               activation codes as E4M3 bytes (the copy the quantiser writes
 //               beside the packed codes) and the prepared E4M3 weight codes,
 //               128 rows x 128 B each, 128-byte swizzled; per tile one stage
-//               of lora_act / L2 (fp32); per group the tile's 128 fp16 s_x
-//               and 128 fp16 s_w into the first K row of a scale slot (four
-//               128-byte bulk copies).
+//               of lora_act / L2 (fp32).
+//   warp 18     scale producer: per group the tile's 128 fp16 s_x and 128
+//               fp16 s_w into the first K row of a scale slot (four 128-byte
+//               bulk copies), eight slots ahead of the MMAs.
 //   warp 1      TMEM owner and MMA issuer: per group two kind::f8f6f4 MMAs
 //               (K = 32) into P and one kind::f16 MMA (K = 16, MN-major
 //               operands from the scale slot) into C, in one of two buffers
@@ -49,12 +50,13 @@ namespace svdq {
 namespace {
 
 constexpr int kTileM = 128, kTileN = 128;
-constexpr int kI4Stages = 6;
+constexpr int kI4Stages = 5;
 constexpr int kA8Bytes = kTileM * 128;   // activation codes of a stage (E4M3): 128 K per row
 constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes (E4M3)
 constexpr int kI4StageBytes = kA8Bytes + kB8Bytes;  // 32 KB
 constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
-constexpr int kI4Threads = 32 * (2 + kI4EpiWarps);
+constexpr int kScaleWarp = 2 + kI4EpiWarps;
+constexpr int kI4Threads = 32 * (3 + kI4EpiWarps);
 constexpr int kAccBufs = 2;      // group buffers of 256 TMEM columns: P (128) then C (128)
 constexpr uint32_t kI4TmemCols = 256 * kAccBufs;
 // Scale slots: the two operands of a group's C MMA, each an MN-major
@@ -62,7 +64,7 @@ constexpr uint32_t kI4TmemCols = 256 * kAccBufs;
 // 0-7); only row 0 of each atom is ever written (the group's scales), rows
 // 1-7 stay zero, and K rows 8-15 of every operand are one shared 2 KB block
 // of zeros (reached through the descriptor's K-group stride).
-constexpr int kScaleSlots = 6;
+constexpr int kScaleSlots = 8;
 constexpr int kSlotBytes = 4096;  // s_x operand (2 KB), then s_w operand (2 KB)
 constexpr int kScaleOff = kI4Stages * kI4StageBytes;
 constexpr int kZeroOff = kScaleOff + kScaleSlots * kSlotBytes;
@@ -170,7 +172,6 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     // ------------------------------------------------ TMA producer (whole warp)
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t sc_count = 0;  // scale slots filled so far
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
       for (int kb = 0; kb < num_kb + p.n_lora; ++kb) {
@@ -191,30 +192,32 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         issued_mask |= 1u << stage;
         issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
         if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
-        // the scales of this stage's groups, one slot per group: row 0 of the
-        // two atoms of each operand (64 fp16 = 128 bytes each)
-        if (kb < num_kb) {
-          const int ng = min(2, groups - 2 * kb);
-          for (int gi = 0; gi < ng; ++gi, ++sc_count) {
-            const uint32_t ss = sc_count % kScaleSlots;
-            const uint32_t sp = (sc_count / kScaleSlots) & 1;
-            if (!mbar_wait_warp(&sc_empty[ss], sp ^ 1, abort_flag)) goto teardown;
-            if (elect_one()) {
-              const int g = 2 * kb + gi;
-              uint8_t* dst = smem + kScaleOff + ss * kSlotBytes;
-              const __half* sxg = p.sx + static_cast<size_t>(g) * p.m_pad + m0;
-              const __half* swg = p.sw + static_cast<size_t>(g) * p.n_pad + n0;
-              mbar_arrive_expect_tx(&sc_full[ss], 512);
-              bulk_load(dst, sxg, 128, &sc_full[ss]);
-              bulk_load(dst + 1024, sxg + 64, 128, &sc_full[ss]);
-              bulk_load(dst + 2048, swg, 128, &sc_full[ss]);
-              bulk_load(dst + 3072, swg + 64, 128, &sc_full[ss]);
-            }
-            __syncwarp();
-            sc_mask |= 1u << ss;
-            sc_par = (sc_par & ~(1u << ss)) | (sp << ss);
-          }
+      }
+    }
+  } else if (warp == kScaleWarp) {
+    // ------------------------------------------ scale producer (whole warp)
+    // one slot per group: row 0 of the two atoms of each operand (64 fp16 =
+    // 128 bytes each)
+    uint32_t sc_count = 0;  // scale slots filled so far
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int m0 = (tile % num_m) * kTileM, n0 = (tile / num_m) * kTileN;
+      for (int g = 0; g < groups; ++g, ++sc_count) {
+        const uint32_t ss = sc_count % kScaleSlots;
+        const uint32_t sp = (sc_count / kScaleSlots) & 1;
+        if (!mbar_wait_warp(&sc_empty[ss], sp ^ 1, abort_flag)) goto teardown;
+        if (elect_one()) {
+          uint8_t* dst = smem + kScaleOff + ss * kSlotBytes;
+          const __half* sxg = p.sx + static_cast<size_t>(g) * p.m_pad + m0;
+          const __half* swg = p.sw + static_cast<size_t>(g) * p.n_pad + n0;
+          mbar_arrive_expect_tx(&sc_full[ss], 512);
+          bulk_load(dst, sxg, 128, &sc_full[ss]);
+          bulk_load(dst + 1024, sxg + 64, 128, &sc_full[ss]);
+          bulk_load(dst + 2048, swg, 128, &sc_full[ss]);
+          bulk_load(dst + 3072, swg + 64, 128, &sc_full[ss]);
         }
+        __syncwarp();
+        sc_mask |= 1u << ss;
+        sc_par = (sc_par & ~(1u << ss)) | (sp << ss);
       }
     }
   } else if (warp == 1) {
@@ -422,6 +425,8 @@ teardown:
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kI4Stages; ++s)
       if (issued_mask & (1u << s)) mbar_wait_limited(&full[s], (issued_par >> s) & 1u, 200000000ull);
+  }
+  if (warp == kScaleWarp && lane == 0) {
     for (int s = 0; s < kScaleSlots; ++s)
       if (sc_mask & (1u << s)) mbar_wait_limited(&sc_full[s], (sc_par >> s) & 1u, 200000000ull);
   }

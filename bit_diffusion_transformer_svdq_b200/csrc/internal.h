@@ -32,7 +32,7 @@ inline size_t int4_q8_offset(int64_t M, int K) { return static_cast<size_t>(roun
 struct WeightLayout {
   size_t qw, sw, l1s, l2, inv_lambda, bias, status, amax, total;
   size_t sw_bytes;
-  size_t qw8, sw32;  // INT4 only (0 otherwise): codes as E4M3 bytes, fp32 group scales
+  size_t qw8;  // INT4 only (0 otherwise): codes as E4M3 bytes
 };
 
 // INT4 working copies for the tensor-core GEMM.  tcgen05 has no 4-bit
@@ -66,7 +66,6 @@ struct svdq_weights {
   uint32_t* amax; // scratch: [0], [1] the preparation's amax and g_w; [2], [3] the activation amax
                   // reduction (max, block count), zero between calls
   uint8_t* qw8;   // INT4: n_pad x K codes as E4M3 bytes (rows past N zero); NVFP4: null
-  float* sw32;    // INT4: [K/64][n_pad] group scales as fp32; NVFP4: null
   int device;
   CUtensorMap tm_qw;  // weight codes, 128-byte swizzled boxes of 128 rows
   CUtensorMap tm_l2;  // fp32 L2, 128-byte swizzled boxes of 128 rows

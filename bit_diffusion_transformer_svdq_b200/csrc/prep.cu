@@ -147,10 +147,10 @@ __global__ void quantize_weights_kernel(const float* __restrict__ W, const float
   }
 }
 
-// INT4 working copies: the codes as E4M3 bytes in natural K order (rows
-// N..n_pad zero) and the group scales as fp32, [K/64][n_pad].
-__global__ void int4_e4m3_kernel(const uint8_t* __restrict__ qw, const __half* __restrict__ sw, int N, int K,
-                                 int64_t n_pad, uint8_t* __restrict__ qw8, float* __restrict__ sw32) {
+// INT4 working copy: the codes as E4M3 bytes in natural K order (rows
+// N..n_pad zero).
+__global__ void int4_e4m3_kernel(const uint8_t* __restrict__ qw, int N, int K, int64_t n_pad,
+                                 uint8_t* __restrict__ qw8) {
   const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
   const size_t blocks = static_cast<size_t>(n_pad) * (K / 8);
   if (i < blocks) {
@@ -171,8 +171,6 @@ __global__ void int4_e4m3_kernel(const uint8_t* __restrict__ qw, const __half* _
     }
     *reinterpret_cast<uint2*>(qw8 + static_cast<size_t>(n) * K + 8 * j) = out;
   }
-  const size_t scales = static_cast<size_t>(K / 64) * n_pad;
-  if (i < scales) sw32[i] = __half2float(sw[i]);
 }
 
 __global__ void l1s_kernel(const uint16_t* __restrict__ L1, const float* __restrict__ inv, int K, int r, int r_pad,
@@ -226,9 +224,8 @@ cudaError_t launch_prepare(const svdq_weights* w, const float* W, const float* l
   } else {
     quantize_weights_kernel<true><<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, s>>>(
         W, lambda, L1, L2, N, K, r, g_w_dev, w->n_pad, w->qw, static_cast<uint8_t*>(w->sw), 0);
-    const size_t work = std::max(static_cast<size_t>(w->n_pad) * (K / 8), static_cast<size_t>(K / 64) * w->n_pad);
-    int4_e4m3_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(
-        w->qw, static_cast<const __half*>(w->sw), N, K, w->n_pad, w->qw8, w->sw32);
+    const size_t work = static_cast<size_t>(w->n_pad) * (K / 8);
+    int4_e4m3_kernel<<<static_cast<unsigned>((work + 255) / 256), 256, 0, s>>>(w->qw, N, K, w->n_pad, w->qw8);
   }
   if (rp > 0) {
     const size_t n1 = static_cast<size_t>(rp) * K;
