@@ -226,30 +226,36 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     uint32_t phase = 0;
     uint32_t gcount = 0;  // buffer uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
     uint32_t sc_use = 0;  // scale slots consumed
-    const uint32_t zero_blk = smem_u32(smem + kZeroOff);
+    // Descriptors move with the slot or stage in their address field only
+    // (and, for the scale operands, the K-group stride to the shared zero
+    // block, which shrinks by as much): one add each.
+    const uint32_t sx0 = smem_u32(smem + kScaleOff), zero_blk = smem_u32(smem + kZeroOff);
+    const uint64_t dsx0 = sdesc_sw128_mn(sx0, 1024, zero_blk - sx0);
+    constexpr uint64_t kSlotStep = (uint64_t(kSlotBytes) >> 4) - ((uint64_t(kSlotBytes) >> 4) << 32);
+    constexpr uint64_t kSwStep = (uint64_t(2048) >> 4) - ((uint64_t(2048) >> 4) << 32);
+    const uint64_t da0 = sdesc_sw128(smem_u32(smem));
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
         tc_fence_after();
-        const uint32_t sa = smem_u32(smem + stage * kI4StageBytes);
-        const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
+        const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
         const int ng = min(2, groups - 2 * kb);
         for (int gi = 0; gi < ng; ++gi, ++gcount, ++sc_use) {
           const uint32_t ss = sc_use % kScaleSlots;
-          if (!mbar_wait_warp(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag)) goto teardown;
           const uint32_t buf = gcount % kAccBufs;
-          if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
+          if (!mbar_wait_warp(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag) ||
+              !mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag))
+            goto teardown;
           tc_fence_after();
           if (elect_one()) {
             const uint32_t d = tmem + buf * 256;
+            const uint64_t dsx = dsx0 + ss * kSlotStep;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // K = 32 E4M3 (32 bytes) per MMA
               mma_f8(d, da + 4 * gi + 2 * k, db + 4 * gi + 2 * k, kIdescF8, k ? 1u : 0u);
             // C = s_x s_w^T: MN-major operands, atoms 1 KB apart along M / N,
             // K rows 8-15 in the shared zero block
-            const uint32_t sxa = smem_u32(smem + kScaleOff + ss * kSlotBytes), swa = sxa + 2048;
-            mma_bf16(d + 128, sdesc_sw128_mn(sxa, 1024, zero_blk - sxa), sdesc_sw128_mn(swa, 1024, zero_blk - swa),
-                     kIdescScale, 0u);
+            mma_bf16(d + 128, dsx, dsx + kSwStep, kIdescScale, 0u);
             tc_commit(&acc_full[buf]);
             tc_commit(&sc_empty[ss]);
           }
@@ -266,8 +272,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
           if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t sa = smem_u32(smem + stage * kI4StageBytes);
-            const uint64_t da = sdesc_sw128(sa), db = sdesc_sw128(sa + kA8Bytes);
+            const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
 #pragma unroll
             for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
               mma_tf32(tmem + buf * 256, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
@@ -307,7 +312,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       const int uses = groups + (p.n_lora > 0 ? 1 : 0);
       for (int g = 0; g < uses; ++g, ++gcount) {
         const uint32_t buf = gcount % kAccBufs;
-        if (!mbar_wait(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_sleep(&acc_full[buf], (gcount / kAccBufs) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tb = tq + buf * 256;
 #pragma unroll
