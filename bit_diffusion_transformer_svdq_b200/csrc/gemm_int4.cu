@@ -24,11 +24,12 @@
 //   warp 18     scale producer: per group the tile's 128 fp16 s_x and 128
 //               fp16 s_w into the first K row of a scale slot (four 128-byte
 //               bulk copies), eight slots ahead of the MMAs.
-//   warp 1      TMEM owner and MMA issuer: per group two kind::f8f6f4 MMAs
-//               (K = 32) into P and one kind::f16 MMA (K = 16, MN-major
-//               operands from the scale slot) into C, in one of two buffers
-//               of 256 columns (P, C); per tile four kind::tf32 MMAs of the
-//               lora-up into the next buffer's P, as one more "group".
+//   warps 1, 19 MMA issuers (warp 1 also owns TMEM), one per buffer: for
+//               the groups whose buffer use is even (warp 1) or odd (warp 19)
+//               two kind::f8f6f4 MMAs (K = 32) into P and one kind::f16 MMA
+//               (K = 16, MN-major operands from the scale slot) into C, the
+//               buffer's 256 columns; per tile four kind::tf32 MMAs of the
+//               lora-up into the next use's P, as one more "group".
 //   warps 2-17  epilogue: warp w owns rows 32 (w % 4) .. + 31 (its TMEM
 //               lane quarter) and columns 32 ((w - 2) / 4) .. + 31; per group
 //               it loads P and C in two halves of 16 columns, frees the
@@ -56,7 +57,8 @@ constexpr int kB8Bytes = kTileN * 128;   // prepared weight codes (E4M3)
 constexpr int kI4StageBytes = kA8Bytes + kB8Bytes;  // 32 KB
 constexpr int kI4EpiWarps = 16;  // 4 lane quarters x 4 column slices of 32
 constexpr int kScaleWarp = 2 + kI4EpiWarps;
-constexpr int kI4Threads = 32 * (3 + kI4EpiWarps);
+constexpr int kMma2Warp = 3 + kI4EpiWarps;  // the second MMA issuer
+constexpr int kI4Threads = 32 * (4 + kI4EpiWarps);
 constexpr int kAccBufs = 2;      // group buffers of 256 TMEM columns: P (128) then C (128)
 constexpr uint32_t kI4TmemCols = 256 * kAccBufs;
 // Scale slots: the two operands of a group's C MMA, each an MN-major
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kI4Stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 2);  // both MMA issuers
     }
     for (int b = 0; b < kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -144,7 +146,7 @@ __global__ void __launch_bounds__(kI4Threads, 1)
       mbar_init(&sc_full[b], 1);
       mbar_init(&sc_empty[b], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,12 +222,19 @@ __global__ void __launch_bounds__(kI4Threads, 1)
         sc_par = (sc_par & ~(1u << ss)) | (sp << ss);
       }
     }
-  } else if (warp == 1) {
-    // --------------------------------------------- MMA issuer (whole warp)
+  } else if (warp == 1 || warp == kMma2Warp) {
+    // -------------------------------------------- MMA issuers (whole warps)
+    // Warp 1 issues the buffer uses of even count (TMEM buffer 0), warp 19
+    // those of odd count (buffer 1): two independent instruction streams
+    // feed the tensor core.  Both walk every ring stage, waiting until it
+    // is full and then releasing it (empty counts both warps); a stage's
+    // group is multiplied by the warp that owns its use.
+    const uint32_t par = warp == 1 ? 0u : 1u;
+    const uint32_t d = tmem + par * 256;
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t gcount = 0;  // buffer uses so far: buffer gcount % kAccBufs, its use gcount / kAccBufs
-    uint32_t sc_use = 0;  // scale slots consumed
+    uint32_t use = 0;     // buffer uses so far, both warps': use u goes to buffer u % 2
+    uint32_t sc_use = 0;  // scale slots consumed so far, both warps'
     // Descriptors move with the slot or stage in their address field only
     // (and, for the scale operands, the K-group stride to the shared zero
     // block, which shrinks by as much): one add each.
@@ -237,18 +246,16 @@ __global__ void __launch_bounds__(kI4Threads, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       for (int kb = 0; kb < num_kb; ++kb) {
         if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
-        tc_fence_after();
-        const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
         const int ng = min(2, groups - 2 * kb);
-        for (int gi = 0; gi < ng; ++gi, ++gcount, ++sc_use) {
-          const uint32_t ss = sc_use % kScaleSlots;
-          const uint32_t buf = gcount % kAccBufs;
-          if (!mbar_wait_warp(&sc_full[ss], (sc_use / kScaleSlots) & 1, abort_flag) ||
-              !mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag))
+        const int gi = static_cast<int>((par ^ use) & 1u);  // the stage's group whose use is this warp's
+        if (gi < ng) {
+          const uint32_t ss = (sc_use + gi) % kScaleSlots;
+          if (!mbar_wait_warp(&sc_full[ss], ((sc_use + gi) / kScaleSlots) & 1, abort_flag) ||
+              !mbar_wait_warp(&acc_empty[par], (((use + gi) >> 1) & 1) ^ 1, abort_flag))
             goto teardown;
           tc_fence_after();
           if (elect_one()) {
-            const uint32_t d = tmem + buf * 256;
+            const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
             const uint64_t dsx = dsx0 + ss * kSlotStep;
 #pragma unroll
             for (int k = 0; k < 2; ++k)  // K = 32 E4M3 (32 bytes) per MMA
@@ -256,34 +263,45 @@ __global__ void __launch_bounds__(kI4Threads, 1)
             // C = s_x s_w^T: MN-major operands, atoms 1 KB apart along M / N,
             // K rows 8-15 in the shared zero block
             mma_bf16(d + 128, dsx, dsx + kSwStep, kIdescScale, 0u);
-            tc_commit(&acc_full[buf]);
+            tc_commit(&acc_full[par]);
             tc_commit(&sc_empty[ss]);
-          }
-          __syncwarp();
-        }
-        if (elect_one()) tc_commit(&empty[stage]);
-        __syncwarp();
-        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
-      }
-      if (p.n_lora > 0) {  // the lora-up as one more buffer use (P only), of scale 1
-        const uint32_t buf = gcount % kAccBufs;
-        if (!mbar_wait_warp(&acc_empty[buf], ((gcount / kAccBufs) & 1) ^ 1, abort_flag)) goto teardown;
-        for (int j = 0; j < p.n_lora; ++j) {
-          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
-          tc_fence_after();
-          if (elect_one()) {
-            const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
-              mma_tf32(tmem + buf * 256, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
             tc_commit(&empty[stage]);
           }
           __syncwarp();
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[stage]);
+        }
+        use += ng;
+        sc_use += ng;
+        if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
+      }
+      if (p.n_lora > 0) {  // the lora-up as one more buffer use (P only), of scale 1
+        const bool own = (use & 1u) == par;
+        if (own && !mbar_wait_warp(&acc_empty[par], ((use >> 1) & 1) ^ 1, abort_flag)) goto teardown;
+        for (int j = 0; j < p.n_lora; ++j) {
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) goto teardown;
+          if (own) {
+            tc_fence_after();
+            if (elect_one()) {
+              const uint64_t da = da0 + static_cast<uint64_t>(stage) * (kI4StageBytes >> 4), db = da + (kA8Bytes >> 4);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)  // K = 8 tf32 (32 bytes) per MMA
+                mma_tf32(d, da + 2 * k, db + 2 * k, kIdescTf32x, (j | k) ? 1u : 0u);
+              tc_commit(&empty[stage]);
+            }
+            __syncwarp();
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+          }
           if (++stage == kI4Stages) { stage = 0; phase ^= 1; }
         }
-        if (elect_one()) tc_commit(&acc_full[buf]);
-        __syncwarp();
-        ++gcount;
+        if (own) {
+          if (elect_one()) tc_commit(&acc_full[par]);
+          __syncwarp();
+        }
+        ++use;
       }
     }
   } else {
@@ -435,7 +453,7 @@ teardown:
     for (int s = 0; s < kScaleSlots; ++s)
       if (sc_mask & (1u << s)) mbar_wait_limited(&sc_full[s], (sc_par >> s) & 1u, 200000000ull);
   }
-  if (warp == 1) {
+  if (warp == 1 || warp == kMma2Warp) {
     if (elect_one()) {
       tc_commit(drain);  // the lane that issued the MMAs: arrives once they have finished
       mbar_wait_limited(drain, 0, 200000000ull);
