@@ -15,14 +15,15 @@
 // X_hat is staged in shared memory as fp32 (one RN32 multiply per element
 // and CTA); reads of it are warp-wide broadcasts.
 //
-// Decoding: a 4-bit two's-complement code v at nibble p (0..3) of a 16-bit
-// half-word h becomes an fp32 without a conversion instruction:
-//     bits((h & (0xF << 4p)) ^ (0x4B000000 | 8 << 4p)) = 2^23 + (v + 8) 16^p,
-// minus (2^23 + 8 * 16^p) is v 16^p exactly.  Each nibble position keeps
-// its own fp32 sum of (v 16^p) x; the powers of two leave the rounding of
-// every product and sum as for v x, and the four sums are folded with
-// exact scalings 16^-p per group before the group scale multiplies them.
-// The 8 warps' partial rows are added in warp order through shared memory.
+// Decoding: a 4-bit two's-complement code v becomes an fp32 without a
+// conversion instruction.  One XOR per 32-bit word of eight codes turns
+// every nibble into v + 8; two masks split the word into the low and the
+// high nibbles of its bytes; a byte permute then puts one of them under the
+// bytes of 0x4B000000, giving bits 0x4B0000(v + 8) = 2^23 + v + 8, and one
+// packed subtraction of 2^23 + 8 leaves v exactly.  Every decoded pair
+// feeds a packed FMA with its two activations; a group's four partial sums
+// are added before the group scale multiplies them, and the 8 warps'
+// partial rows are added in warp order through shared memory.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -50,6 +51,8 @@ __global__ void __launch_bounds__(kAwqThreads)
   const int n = nb * 32 + lane;  // < n_pad: padding rows hold zero codes and scales
   const int groups = K / 64;
   const uint8_t* tile = qg + static_cast<size_t>(nb) * (K / 32) * 512 + lane * 16;
+  // the upper three bytes of 2^23 as fp32, in a register for the byte permutes
+  const uint32_t kMagic = 0x4B000000u;
   float y[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) y[m] = 0.0f;
@@ -101,35 +104,35 @@ __global__ void __launch_bounds__(kAwqThreads)
         if (it + kD < iters) load(d, it + kD);
         const int g = warp + kAwqWarps * it;
         const uint32_t words[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        // nibble positions (0, 1) and (2, 3) of a half-word as fp32 pairs
-        // (packed two-wide adds and FMAs)
-        const float2 kC01 = make_float2(-(8388608.0f + 8.0f), -(8388608.0f + 128.0f));
-        const float2 kC23 = make_float2(-(8388608.0f + 2048.0f), -(8388608.0f + 32768.0f));
-        float2 a01[MT], a23[MT];
+        const float2 kOff = make_float2(-(8388608.0f + 8.0f), -(8388608.0f + 8.0f));
+        float2 a0[MT], a1[MT];  // codes of bytes 0, 2 and of bytes 1, 3 of every word
 #pragma unroll
-        for (int m = 0; m < MT; ++m) a01[m] = a23[m] = make_float2(0.0f, 0.0f);
+        for (int m = 0; m < MT; ++m) a0[m] = a1[m] = make_float2(0.0f, 0.0f);
 #pragma unroll
-        for (int wd = 0; wd < 8; ++wd) {  // 8 codes: k = 64 g + 8 wd + (0..7)
+        for (int wd = 0; wd < 8; ++wd) {  // 8 codes: k = 64 g + 8 wd + (0..7), low nibble = even k
+          const uint32_t wq = words[wd] ^ 0x88888888u;    // every nibble v -> v + 8
+          const uint32_t lo = wq & 0x0F0F0F0Fu;            // byte j: code 2j
+          const uint32_t hi = (wq >> 4) & 0x0F0F0F0Fu;     // byte j: code 2j + 1
+          const int k = 64 * g + 8 * wd;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const uint32_t h = half ? (words[wd] >> 16) : words[wd];
-            const int k = 64 * g + 8 * wd + 4 * half;
-            const float2 v01 = __fadd2_rn(make_float2(__uint_as_float((h & 0xFu) ^ 0x4B000008u),
-                                                      __uint_as_float((h & 0xF0u) ^ 0x4B000080u)), kC01);
-            const float2 v23 = __fadd2_rn(make_float2(__uint_as_float((h & 0xF00u) ^ 0x4B000800u),
-                                                      __uint_as_float((h & 0xF000u) ^ 0x4B008000u)), kC23);
+          for (int jj = 0; jj < 4; jj += 2) {  // bytes jj, jj + 1: codes k + 2 jj .. k + 2 jj + 3
+            const float2 v0 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, kMagic, 0x7650u + jj)),
+                                                     __uint_as_float(__byte_perm(hi, kMagic, 0x7650u + jj))),
+                                         kOff);
+            const float2 v1 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, kMagic, 0x7651u + jj)),
+                                                     __uint_as_float(__byte_perm(hi, kMagic, 0x7651u + jj))),
+                                         kOff);
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
-              const float4 x = *reinterpret_cast<const float4*>(xs + m * K + k);  // broadcast
-              a01[m] = __ffma2_rn(v01, make_float2(x.x, x.y), a01[m]);
-              a23[m] = __ffma2_rn(v23, make_float2(x.z, x.w), a23[m]);
+              const float4 x = *reinterpret_cast<const float4*>(xs + m * K + k + 2 * jj);  // broadcast
+              a0[m] = __ffma2_rn(v0, make_float2(x.x, x.y), a0[m]);
+              a1[m] = __ffma2_rn(v1, make_float2(x.z, x.w), a1[m]);
             }
           }
         }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const float gsum = __fadd_rn(__fadd_rn(a01[m].x, __fmul_rn(a01[m].y, 0.0625f)),
-                                       __fadd_rn(__fmul_rn(a23[m].x, 0.00390625f), __fmul_rn(a23[m].y, 0.000244140625f)));
+          const float gsum = __fadd_rn(__fadd_rn(a0[m].x, a0[m].y), __fadd_rn(a1[m].x, a1[m].y));
           y[m] = __fmaf_rn(s, gsum, y[m]);
         }
       }
