@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(kAwqThreads)
   // the next kD groups are in flight while one is decoded (rotating slots).
   // The first loads are issued before X_hat is staged, so that their
   // latency overlaps it.
-  constexpr int kD = 4;
+  constexpr int kD = 2;
   const int iters = groups > warp ? (groups - warp + kAwqWarps - 1) / kAwqWarps : 0;
   uint4 ca[kD], cb[kD];
   float sc[kD];
