@@ -57,6 +57,28 @@ def test_noalloc_forward_matches_workspace_forward_twice(svdq):
     assert svdq.svdq_device_status(w) == 0
 
 
+def test_noalloc_int4_matches_workspace_forward(svdq):
+    """INT4 weights: the scratch also holds the E4M3 copy of the codes that
+    the GEMM reads.  Two calls (the second with fewer rows, over the first's
+    leftovers) equal the workspace forward bit for bit."""
+    K, N = 576, 320  # an odd number of 64-groups, a ragged last column tile
+    li = synth.make_layer("int4", 41, M=300, K=K, N=N)
+    ol = T.oracle_layer(li, precision="int4")
+    w = T.gpu_prepare(svdq, li, ol, "int4")
+    x2 = synth.make_layer("int4", 42, M=130, K=K, N=N).x_bits
+    for call, x_bits in enumerate((li.x_bits, x2)):
+        M = x_bits.shape[0]
+        ws = T.aligned_empty(svdq.svdq_workspace_bytes(w, M))
+        X = T.dev_u16(x_bits)
+        ref = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        svdq.svdq_linear_forward(w, X, M, 1.0, ref, ws, ws.numel(), svdq.SVDQ_OUT_F32)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        svdq.svdq_linear_forward_noalloc(w, X, M, 1.0, y, svdq.SVDQ_OUT_F32)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), call
+    assert svdq.svdq_device_status(w) == 0
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch(svdq):
     li = synth.make_layer("tiny", 3, K=3072, N=256, M=16)
     ol = T.oracle_layer(li)
