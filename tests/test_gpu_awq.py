@@ -56,6 +56,10 @@ CASES = [
     ("m3", dict(M=3, K=512, N=256)),
     ("m9_two_row_blocks", dict(M=9, K=1024, N=96)),
     ("m5", dict(M=5, K=256, N=512)),
+    # long K: 24 groups per warp, so the rotating prefetch slots wrap many
+    # times; four activation rows per CTA with a ragged last row block
+    ("m1_long_k", dict(M=1, K=12288, N=128)),
+    ("m4_long_k_ragged_n", dict(M=4, K=6144, N=208)),
 ]
 
 
@@ -80,7 +84,7 @@ def test_awq_parity(svdq, name, over, out_dtype):
     X = T.dev_u16(li.x_bits)
     Y = torch.empty((M, N), dtype=torch.float32 if out_dtype == 1 else torch.bfloat16, device="cuda")
     svdq.svdq_awq_w4a16_forward(w, X, M, Y, out_dtype)
-    torch.cuda.synchronize()
+    assert svdq.svdq_device_status(w) == 0
     y = Y.float().cpu().numpy()
     ref = A.forward(li.x, prep)
     xh = (li.x * prep.inv_alpha[None, :]).astype(np.float32)
