@@ -22,7 +22,8 @@ equivalent operations per second over the step's linears, the low-rank
 flops not counted) summed over all ranks; ranks run independent replicas
 (the layer has no exchange step).  L2 is flushed before every timed step by
 reading a 256 MiB buffer (a read leaves only clean lines, so the step pays
-no write-back of the flush), outside the step's CUDA-event bracket.
+no write-back of the flush), outside the step's CUDA-event bracket;
+`--flush-mib` sets its size (0 skips it: a warm-L2 diagnostic).
 `--impl reference` times the CPU oracle on the host cores on a bounded row
 sample of the same workload.
 """
@@ -250,7 +251,7 @@ def run_layers(args, rank, world, local_rank):
     desc, lis = _layer_inputs(args)
     _, specs = LAYER_WORKLOADS[args.workload]
     layers = [_gpu_layer(svdq, li, dev, seed) for li, (_, seed) in zip(lis, specs)]
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    flush = _make_flush(args, dev)
     pro = None
     if args.qkv_prologue:  # the fused attention prologue: seeded QK-norm weights and rotary tables
         if args.workload != "qkv":
@@ -426,7 +427,7 @@ def run_layers(args, rank, world, local_rank):
             "data": "synthetic",
             "config": {"workload": f"{args.workload}: {desc}",
                        "linears": [f"{L['name']} M={L['M']} K={L['K']} N={L['N']}" for L in layers],
-                       "l2": "flushed (256 MiB read) before each step, outside the step's event bracket",
+                       "l2": _l2_note(args),
                        "parallelism": f"replicas x{world}"},
             "roofline": roof,
             "roofline_quantize": roof_q,
@@ -507,7 +508,7 @@ def run_stack(args, rank, world, local_rank):
     ws_bytes = max(svdq.svdq_workspace_bytes(w, M) for (w, _, _, _, _) in layers[:4])
     ws = svdq.alloc_workspace(layers[0][0], M, dev, nbytes=ws_bytes)
     Ys = {N: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for (_, _, _, N, _) in layers[:4]}
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    flush = _make_flush(args, dev)
 
     words = torch.zeros(2, dtype=torch.float32, device=dev)
     epis = {}
@@ -568,7 +569,7 @@ def run_stack(args, rank, world, local_rank):
             "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
             "config": {"workload": f"{args.blocks} blocks x 4 linears (QKV, out, MLP up, down), M={M}, rank 32, nvfp4",
                        "linears": len(layers), "tensor_scale": args.scale,
-                       "l2": "flushed (256 MiB read) once before each step",
+                       "l2": _l2_note(args, "once before each step"),
                        "parallelism": f"replicas x{world}"},
             "gpu_launches": per_step * args.steps, "clocks": clocks}), flush=True)
 
@@ -596,7 +597,7 @@ def run_awq(args, rank, world, local_rank):
     del W
     X = torch.from_numpy(li.x_bits.view(np.int16)).to(dev)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    flush = _make_flush(args, dev)
     for _ in range(args.warmup):
         flush.sum()
         svdq.svdq_awq_w4a16_forward(w, X, M, Y, svdq.SVDQ_OUT_BF16, stream)
@@ -629,11 +630,31 @@ def run_awq(args, rank, world, local_rank):
             "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int4 weights x fp32 (bf16 activations)", "data": "synthetic",
             "config": {"workload": f"awq adaLN modulation M={M} K={K} N={N} int4/64",
-                       "l2": "flushed (256 MiB read) before each step", "parallelism": f"replicas x{world}"},
+                       "l2": _l2_note(args, "before each step"), "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "kernel": "awq_gemv_kernel", "achieved": gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"], "traffic": None,
                          "algorithmic_bytes": nbytes, "peak_source": f"{peak_kind} hbm_gbs"},
             "gpu_launches": args.steps, "clocks": clocks}), flush=True)
+
+
+class _NoFlush:
+    def sum(self):
+        return None
+
+
+def _make_flush(args, dev):
+    """The L2 read-flush run before every step: a buffer of --flush-mib MiB
+    that is summed (0: no flush, a warm-L2 diagnostic only)."""
+    import torch
+    if args.flush_mib <= 0:
+        return _NoFlush()
+    return torch.ones(args.flush_mib << 18, dtype=torch.float32, device=dev)
+
+
+def _l2_note(args, when="before each step, outside the step's event bracket"):
+    if args.flush_mib <= 0:
+        return "not flushed (warm-L2 diagnostic, not a bench value)"
+    return f"flushed ({args.flush_mib} MiB read) {when}"
 
 
 def _job_tops(ops_per_rank, t_ms_max, world):
@@ -665,6 +686,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-mib", type=int, default=256,
+                    help="MiB read before every step to flush the L2 (0: none, a warm-L2 diagnostic)")
     ap.add_argument("--rows", type=int, default=None, help="override M (smaller profiling cases only)")
     ap.add_argument("--workload", default="mlp", choices=["mlp", "qkv", "int4", "tiny", "stack", "awq"],
                     help="mlp (default): the FLUX MLP pair; qkv: the fused QKV projection; int4: the INT4 "
